@@ -1,0 +1,144 @@
+"""fp64 CPU oracle of the 2D selective-scan forward (2DMamba), as a ctypes binding.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` may import this package.  The product path (the CUDA
+library under ``selective_state_space_scan2d_b200``) shares no code with it.
+
+The arithmetic lives in ``scan2d_oracle.c`` (plain single-threaded C, fp64), written
+from the recurrences on the pages ("2DMamba 精读：从小白到博士", section 4.5 (1)
+horizontal scan, (2) vertical scan and output).  This module only builds it with gcc and
+marshals numpy arrays.
+
+Input conventions (numpy):
+  * fp32 tensors are ``float32`` arrays; bf16 tensors are ``uint16`` arrays holding the
+    bf16 bit patterns (numpy has no bf16 dtype).  Every stored value is widened exactly.
+  * x, delta: (batch, channels, H, W); A: (channels, N) float32; B, C: (batch, K, N, H, W);
+    Dskip: (channels,) float32 or None.
+  * ``orient_mask``: bit 0 top-left, bit 1 top-right (flip W), bit 2 bottom-left (flip H),
+    bit 3 bottom-right (flip both).  K = number of set bits.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "scan2d_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle_scan2d.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (plain C99, -O2, no fast-math) into this folder."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-std=c99", "-O2", "-fPIC", "-shared", "-fno-fast-math",
+                               "-ffp-contract=off", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def load_library(path: str | None = None):
+    """ctypes handle of the oracle library (the default build, or another build at path)."""
+    global _lib
+    if path is None and _lib is not None:
+        return _lib
+    lib = ctypes.CDLL(path or build())
+    vp, fp, dp, ip = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
+    i, u = ctypes.c_int, ctypes.c_uint
+    common = [vp, vp, fp, vp, vp, fp, dp, i, i, i, i, i, i, u]
+    lib.scan2d_oracle_fwd.argtypes = common
+    lib.scan2d_oracle_fwd.restype = i
+    lib.scan2d_oracle_maps.argtypes = common + [ip, i]
+    lib.scan2d_oracle_maps.restype = i
+    lib.scan2d_oracle_points.argtypes = common + [ip, i]
+    lib.scan2d_oracle_points.restype = i
+    lib.scan2d_oracle_version.argtypes = []
+    lib.scan2d_oracle_version.restype = i
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _load(lib=None):
+    return lib if lib is not None else load_library()
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _prepare(x, delta, A, B, C, Dskip, orient_mask):
+    x = np.ascontiguousarray(x)
+    delta = np.ascontiguousarray(delta)
+    B = np.ascontiguousarray(B)
+    C = np.ascontiguousarray(C)
+    A = np.ascontiguousarray(A, dtype=np.float32)
+    if Dskip is not None:
+        Dskip = np.ascontiguousarray(Dskip, dtype=np.float32)
+    if x.dtype == np.uint16:
+        is_bf16 = 1
+    elif x.dtype == np.float32:
+        is_bf16 = 0
+    else:
+        raise TypeError("x must be float32 or uint16 (bf16 bits)")
+    for name, t in (("delta", delta), ("B", B), ("C", C)):
+        if t.dtype != x.dtype:
+            raise TypeError(f"{name} must have the dtype of x")
+    batch, channels, H, W = x.shape
+    if delta.shape != x.shape:
+        raise ValueError("delta must have the shape of x")
+    K = bin(orient_mask & 0xF).count("1")
+    if B.ndim == 4:                      # (batch, N, H, W) is the K = 1 layout
+        B = B.reshape(B.shape[0], 1, *B.shape[1:])
+        C = C.reshape(C.shape[0], 1, *C.shape[1:])
+    if B.shape[0] != batch or B.shape[1] != K or B.shape[3:] != (H, W) or C.shape != B.shape:
+        raise ValueError(f"B, C must be (batch, K={K}, N, H, W); got {B.shape}, {C.shape}")
+    N = B.shape[2]
+    if A.shape != (channels, N):
+        raise ValueError("A must be (channels, N)")
+    if Dskip is not None and Dskip.shape != (channels,):
+        raise ValueError("Dskip must be (channels,)")
+    return x, delta, A, B, C, Dskip, (batch, channels, H, W, N, is_bf16)
+
+
+def scan2d_fwd(x, delta, A, B, C, Dskip=None, orient_mask: int = 1, lib=None) -> np.ndarray:
+    """Full fp64 output y (batch, channels, H, W)."""
+    x, delta, A, B, C, Dskip, dims = _prepare(x, delta, A, B, C, Dskip, orient_mask)
+    y = np.empty(x.shape, dtype=np.float64)
+    rc = _load(lib).scan2d_oracle_fwd(_ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(Dskip),
+                                   _ptr(y), *dims, orient_mask)
+    if rc:
+        raise RuntimeError(f"oracle error {rc}")
+    return y
+
+
+def scan2d_maps(x, delta, A, B, C, Dskip, maps, orient_mask: int = 1, lib=None) -> np.ndarray:
+    """fp64 output of the listed (b, d) maps only: shape (len(maps), H, W)."""
+    x, delta, A, B, C, Dskip, dims = _prepare(x, delta, A, B, C, Dskip, orient_mask)
+    m = np.ascontiguousarray(np.asarray(maps, dtype=np.int32).reshape(-1, 2))
+    y = np.empty((m.shape[0], dims[2], dims[3]), dtype=np.float64)
+    rc = _load(lib).scan2d_oracle_maps(_ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(Dskip),
+                                    _ptr(y), *dims, orient_mask, _ptr(m), m.shape[0])
+    if rc:
+        raise RuntimeError(f"oracle error {rc}")
+    return y
+
+
+def scan2d_points(x, delta, A, B, C, Dskip, points, orient_mask: int = 1, lib=None) -> np.ndarray:
+    """fp64 output at the listed (b, d, i, j) positions only."""
+    x, delta, A, B, C, Dskip, dims = _prepare(x, delta, A, B, C, Dskip, orient_mask)
+    p = np.ascontiguousarray(np.asarray(points, dtype=np.int32).reshape(-1, 4))
+    y = np.empty(p.shape[0], dtype=np.float64)
+    rc = _load(lib).scan2d_oracle_points(_ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+                                      _ptr(Dskip), _ptr(y), *dims, orient_mask, _ptr(p), p.shape[0])
+    if rc:
+        raise RuntimeError(f"oracle error {rc}")
+    return y
+
+
+def version() -> int:
+    return _load().scan2d_oracle_version()

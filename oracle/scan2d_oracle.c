@@ -1,0 +1,262 @@
+/*
+ * scan2d_oracle.c -- plain, slow, fp64 reference of the 2D selective-scan forward.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the CPU-baseline
+ * leg of the benchmark may load this code.  The product path (the CUDA library) shares
+ * no code with it and never calls it.
+ *
+ * Sources (web pages on 2DMamba, arXiv 2412.00678):
+ *   [J]  "2DMamba 精读：从小白到博士，彻底拆解 2DMamba" (juejin.cn)
+ *          4.4  "2DMamba 的核心：二维 selective scan"   -- 1D recurrence h_t = A_t h_{t-1} + B_t x_t
+ *          4.5  "2DMamba 如何扩展到二维？" (1) 横向扫描 -- horizontal recurrence
+ *                                         (2) 纵向扫描 -- vertical recurrence, output y = C h
+ *          5.3  "数学层面的关键理解"                    -- unrolled (Manhattan) form
+ *   [PN] papernotes.org notes on the CVPR 2025 paper, "关键设计" (2D selective SSM
+ *          architecture; the 3x3 example; the hardware-aware operator)
+ *
+ * What is computed, for every (b, d) map and every state n (readings of the pages that
+ * are not printed there are marked READING):
+ *   Abar[i,j]  = exp(delta[i,j] * A[d,n])                       READING: zero-order exp,
+ *   Bbar[i,j]  = delta[i,j] * B[n,i,j]                           simplified Euler Bbar
+ *   hh[i,j]    = Abar[i,j]*hh[i,j-1] + Bbar[i,j]*x[i,j]          [J 4.5(1)], hh[i,-1] = 0
+ *   h[i,j]     = Abar[i,j]*h[i-1,j]  + hh[i,j]                   [J 4.5(2)], h[-1,j]  = 0
+ *   y[i,j]    += C[n,i,j]*h[i,j]                                 [J 4.5(2)] output
+ * and finally y[i,j] += Dskip[d]*x[i,j] once (READING: the skip term is not on the pages).
+ * The same Abar is used in both scans and the vertical scan adds no second Bbar
+ * ([J 4.5(2)] writes Abar_{i,j} and h^hor_{i,j} only).
+ *
+ * Orientations (READING of "reverse scans" in [PN 局限与展望] and "四象限" in [J 7.4]):
+ * an orientation flips the map in H and/or W, runs the scan above from its own corner
+ * with its own B_k, C_k (stored in the original, unflipped coordinates), and its output is
+ * added at the original positions.  Bit 0 = top-left (no flip), bit 1 = top-right (flip
+ * W), bit 2 = bottom-left (flip H), bit 3 = bottom-right (both).  delta and A are shared.
+ *
+ * Layouts (all dense, row-major, W fastest):
+ *   x, delta : (batch, channels, H, W)      fp32 or bf16 bits
+ *   A        : (channels, N)                fp32
+ *   B, C     : (batch, K, N, H, W)          fp32 or bf16 bits, K = number of orientations
+ *   Dskip    : (channels)                   fp32, NULL means 0
+ *   y        : (batch, channels, H, W)      fp64 (output of this file)
+ * Every stored input value is converted exactly to double before use.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_VERSION 1
+
+/* bf16 bits -> double, exact (a bf16 value is the top 16 bits of an IEEE fp32 value). */
+static double bf16_to_double(uint16_t v)
+{
+    uint32_t u = ((uint32_t)v) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Element e of a buffer holding fp32 (is_bf16 == 0) or bf16 bits (is_bf16 != 0). */
+static double load(const void *buf, size_t e, int is_bf16)
+{
+    if (is_bf16)
+        return bf16_to_double(((const uint16_t *)buf)[e]);
+    return (double)((const float *)buf)[e];
+}
+
+typedef struct {
+    const void *x, *delta, *B, *C;
+    const float *A, *Dskip;
+    int batch, channels, H, W, N, K, is_bf16;
+} problem;
+
+/* Orientation number (0..3) of the k-th set bit of the mask, or -1. */
+static int orientation_of(unsigned mask, int k)
+{
+    int seen = 0;
+    for (int o = 0; o < 4; ++o) {
+        if (mask & (1u << o)) {
+            if (seen == k)
+                return o;
+            ++seen;
+        }
+    }
+    return -1;
+}
+
+/*
+ * One orientation of one (b, d) map, scanned over the sub-rectangle of scan-order rows
+ * 0..rows-1 and scan-order columns 0..cols-1.  Scan-order (ii, jj) maps to the original
+ * position (flipH ? H-1-ii : ii, flipW ? W-1-jj : jj).  The result C.h is added into
+ * yacc (an H*W array in original coordinates).  hcol is scratch of length >= cols.
+ */
+static void scan_one_orientation(const problem *p, int b, int d, int k, int orient,
+                                 int rows, int cols, double *yacc, double *hcol)
+{
+    const int H = p->H, W = p->W, N = p->N, K = p->K;
+    const int flipW = orient & 1, flipH = (orient >> 1) & 1;
+    const size_t map = ((size_t)b * p->channels + d) * (size_t)H * W;
+    for (int n = 0; n < N; ++n) {
+        const double An = (double)p->A[(size_t)d * N + n];
+        const size_t bc = (((size_t)b * K + k) * N + n) * (size_t)H * W;
+        for (int jj = 0; jj < cols; ++jj)
+            hcol[jj] = 0.0;                                /* h[-1, j] = 0 */
+        for (int ii = 0; ii < rows; ++ii) {
+            const int i = flipH ? H - 1 - ii : ii;
+            double hh = 0.0;                               /* hh[i, -1] = 0 */
+            for (int jj = 0; jj < cols; ++jj) {
+                const int j = flipW ? W - 1 - jj : jj;
+                const size_t pos = (size_t)i * W + j;
+                const double dl = load(p->delta, map + pos, p->is_bf16);
+                const double xv = load(p->x, map + pos, p->is_bf16);
+                const double Bv = load(p->B, bc + pos, p->is_bf16);
+                const double Cv = load(p->C, bc + pos, p->is_bf16);
+                const double abar = exp(dl * An);          /* Abar = exp(delta*A)   */
+                hh = abar * hh + (dl * Bv) * xv;           /* horizontal, [J 4.5(1)] */
+                hcol[jj] = abar * hcol[jj] + hh;           /* vertical,   [J 4.5(2)] */
+                yacc[pos] += Cv * hcol[jj];                /* y = C h,    [J 4.5(2)] */
+            }
+        }
+    }
+}
+
+static int check(const problem *p, unsigned mask)
+{
+    if (!p->x || !p->delta || !p->A || !p->B || !p->C)
+        return -1;
+    if (p->batch < 1 || p->channels < 1 || p->H < 1 || p->W < 1 || p->N < 1)
+        return -2;
+    if (mask == 0 || (mask & ~0xFu))
+        return -4;
+    return 0;
+}
+
+static void init_problem(problem *p, const void *x, const void *delta, const float *A,
+                         const void *B, const void *C, const float *Dskip, int batch,
+                         int channels, int H, int W, int N, int is_bf16, unsigned mask)
+{
+    p->x = x; p->delta = delta; p->A = A; p->B = B; p->C = C; p->Dskip = Dskip;
+    p->batch = batch; p->channels = channels; p->H = H; p->W = W; p->N = N;
+    p->is_bf16 = is_bf16;
+    p->K = 0;
+    for (int o = 0; o < 4; ++o)
+        p->K += (mask >> o) & 1u;
+}
+
+/* y for the maps listed in maps[2*m] = b, maps[2*m+1] = d; y_out is (nmaps, H, W). */
+int scan2d_oracle_maps(const void *x, const void *delta, const float *A, const void *B,
+                       const void *C, const float *Dskip, double *y_out, int batch,
+                       int channels, int H, int W, int N, int is_bf16, unsigned orient_mask,
+                       const int *maps, int nmaps)
+{
+    problem p;
+    init_problem(&p, x, delta, A, B, C, Dskip, batch, channels, H, W, N, is_bf16, orient_mask);
+    int rc = check(&p, orient_mask);
+    if (rc)
+        return rc;
+    if (!y_out || (nmaps > 0 && !maps))
+        return -1;
+    double *hcol = (double *)malloc(sizeof(double) * (size_t)W);
+    if (!hcol)
+        return -8;
+    const size_t HW = (size_t)H * W;
+    for (int m = 0; m < nmaps; ++m) {
+        const int b = maps[2 * m], d = maps[2 * m + 1];
+        if (b < 0 || b >= batch || d < 0 || d >= channels) {
+            free(hcol);
+            return -2;
+        }
+        double *ym = y_out + (size_t)m * HW;
+        const size_t map = ((size_t)b * channels + d) * HW;
+        const double Dd = Dskip ? (double)Dskip[d] : 0.0;
+        for (size_t pos = 0; pos < HW; ++pos)
+            ym[pos] = 0.0;
+        for (int k = 0; k < p.K; ++k)
+            scan_one_orientation(&p, b, d, k, orientation_of(orient_mask, k), H, W, ym, hcol);
+        for (size_t pos = 0; pos < HW; ++pos)                     /* + Dskip * x, once */
+            ym[pos] += Dd * load(x, map + pos, is_bf16);
+    }
+    free(hcol);
+    return 0;
+}
+
+/* y for every map; y_out is (batch, channels, H, W). */
+int scan2d_oracle_fwd(const void *x, const void *delta, const float *A, const void *B,
+                      const void *C, const float *Dskip, double *y_out, int batch,
+                      int channels, int H, int W, int N, int is_bf16, unsigned orient_mask)
+{
+    if (batch < 1 || channels < 1)
+        return -2;
+    int *maps = (int *)malloc(sizeof(int) * 2 * (size_t)batch * channels);
+    if (!maps)
+        return -8;
+    for (int b = 0, m = 0; b < batch; ++b)
+        for (int d = 0; d < channels; ++d, ++m) {
+            maps[2 * m] = b;
+            maps[2 * m + 1] = d;
+        }
+    int rc = scan2d_oracle_maps(x, delta, A, B, C, Dskip, y_out, batch, channels, H, W, N,
+                                is_bf16, orient_mask, maps, batch * channels);
+    free(maps);
+    return rc;
+}
+
+/*
+ * y at single positions.  points[4*q .. 4*q+3] = (b, d, i, j).  Only the rectangle between
+ * each orientation's starting corner and (i, j) can reach (i, j), so the scan runs over
+ * that rectangle alone: the same recurrences, cut short.
+ */
+int scan2d_oracle_points(const void *x, const void *delta, const float *A, const void *B,
+                         const void *C, const float *Dskip, double *y_out, int batch,
+                         int channels, int H, int W, int N, int is_bf16, unsigned orient_mask,
+                         const int *points, int npoints)
+{
+    problem p;
+    init_problem(&p, x, delta, A, B, C, Dskip, batch, channels, H, W, N, is_bf16, orient_mask);
+    int rc = check(&p, orient_mask);
+    if (rc)
+        return rc;
+    if (!y_out || (npoints > 0 && !points))
+        return -1;
+    double *hcol = (double *)malloc(sizeof(double) * (size_t)W);
+    double *yacc = (double *)malloc(sizeof(double) * (size_t)H * W);
+    if (!hcol || !yacc) {
+        free(hcol);
+        free(yacc);
+        return -8;
+    }
+    for (int q = 0; q < npoints; ++q) {
+        const int b = points[4 * q], d = points[4 * q + 1];
+        const int i = points[4 * q + 2], j = points[4 * q + 3];
+        if (b < 0 || b >= batch || d < 0 || d >= channels || i < 0 || i >= H || j < 0 || j >= W) {
+            free(hcol);
+            free(yacc);
+            return -2;
+        }
+        const size_t pos = (size_t)i * W + j;
+        double total = 0.0;
+        for (int k = 0; k < p.K; ++k) {
+            const int o = orientation_of(orient_mask, k);
+            const int flipW = o & 1, flipH = (o >> 1) & 1;
+            const int rows = flipH ? H - i : i + 1;
+            const int cols = flipW ? W - j : j + 1;
+            yacc[pos] = 0.0;
+            /* positions other than (i, j) inside the rectangle also get written; only
+               (i, j) is read, so they are cleared lazily by writing the whole rectangle. */
+            for (int ii = 0; ii < rows; ++ii) {
+                const int ri = flipH ? H - 1 - ii : ii;
+                for (int jj = 0; jj < cols; ++jj)
+                    yacc[(size_t)ri * W + (flipW ? W - 1 - jj : jj)] = 0.0;
+            }
+            scan_one_orientation(&p, b, d, k, o, rows, cols, yacc, hcol);
+            total += yacc[pos];
+        }
+        const size_t map = ((size_t)b * channels + d) * (size_t)H * W;
+        total += (Dskip ? (double)Dskip[d] : 0.0) * load(x, map + pos, is_bf16);
+        y_out[q] = total;
+    }
+    free(hcol);
+    free(yacc);
+    return 0;
+}
+
+int scan2d_oracle_version(void) { return ORACLE_VERSION; }

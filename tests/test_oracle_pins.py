@@ -1,0 +1,325 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself.
+
+Each pin is an independent route to the same number:
+  * the unrolled closed form (a sum over source positions of path products), by brute
+    force on small maps ("2DMamba 精读", section 五.3; product form for varying Abar);
+  * the two scans written as lower-triangular linear systems and solved by LAPACK;
+  * the Manhattan-distance form for constant Abar, and the pages' 3x3 worked example;
+  * the 1D Mamba recurrence when H = 1 or W = 1 ("2DMamba 精读", section 四.4);
+  * linearity in x, B = 0, C picking one state, and orientations as flips of the input.
+A last test plants plausible mistakes in a copy of the oracle and checks that every one
+of them is caught by at least one pin.
+"""
+import json
+import os
+import subprocess
+
+import numpy as np
+import pytest
+
+from selective_state_space_scan2d_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _f64(a):
+    if a.dtype == np.uint16:
+        return inputs.bf16_bits_to_f32(a).astype(np.float64)
+    return a.astype(np.float64)
+
+
+# ----------------------------------------------------------------------------------------
+# independent routes
+# ----------------------------------------------------------------------------------------
+def closed_form_map(x, dl, A, B, C, D):
+    """One map, one orientation (top-left), brute force over all source positions:
+    h[i,j] = sum_{i'<=i, j'<=j} prod_{k=i'+1..i} Abar[k,j] * prod_{l=j'+1..j} Abar[i',l]
+             * Bbar[i',j'] x[i',j'];   y = sum_n C[n] h[n] + D x."""
+    H, W = x.shape
+    y = D * x.copy()
+    for n in range(A.shape[0]):
+        a = np.exp(dl * A[n])
+        u = dl * B[n] * x
+        for i in range(H):
+            for j in range(W):
+                s = 0.0
+                for ip in range(i + 1):
+                    down = np.prod(a[ip + 1:i + 1, j])
+                    for jp in range(j + 1):
+                        right = np.prod(a[ip, jp + 1:j + 1])
+                        s += down * right * u[ip, jp]
+                y[i, j] += C[n, i, j] * s
+    return y
+
+
+def linsolve_map(x, dl, A, B, C, D):
+    """One map, top-left: hh = M_h^{-1} u and h = M_v^{-1} hh with
+    M_h = I - diag(Abar) S_left and M_v = I - diag(Abar) S_up, solved by numpy.linalg."""
+    H, W = x.shape
+    L = H * W
+    y = (D * x).ravel().copy()
+    for n in range(A.shape[0]):
+        a = np.exp(dl * A[n]).ravel()
+        u = (dl * B[n] * x).ravel()
+        Mh = np.eye(L)
+        Mv = np.eye(L)
+        for p in range(L):
+            i, j = divmod(p, W)
+            if j > 0:
+                Mh[p, p - 1] = -a[p]
+            if i > 0:
+                Mv[p, p - W] = -a[p]
+        h = np.linalg.solve(Mv, np.linalg.solve(Mh, u))
+        y += C[n].ravel() * h
+    return y.reshape(H, W)
+
+
+def recurrence_1d(a, u):
+    """Textbook 1D selective recurrence h_t = a_t h_{t-1} + u_t, h_{-1} = 0."""
+    h = np.zeros_like(u)
+    prev = 0.0
+    for t in range(u.shape[0]):
+        prev = a[t] * prev + u[t]
+        h[t] = prev
+    return h
+
+
+def _small(name="tiny", seed=0, **kw):
+    w = inputs.WORKLOADS[name].scaled(**kw)
+    return inputs.make_inputs(w, seed)
+
+
+def _map_args(d, b, ch, k=0):
+    x = _f64(d["x"][b, ch])
+    dl = _f64(d["delta"][b, ch])
+    A = d["A"][ch].astype(np.float64)
+    B = _f64(d["B"][b, k])
+    C = _f64(d["C"][b, k])
+    D = 0.0 if d["Dskip"] is None else float(d["Dskip"][ch])
+    return x, dl, A, B, C, D
+
+
+def _fwd(oracle_mod, d, lib=None, mask=None):
+    return oracle_mod.scan2d_fwd(d["x"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"],
+                                 d["orient_mask"] if mask is None else mask, lib=lib)
+
+
+# ----------------------------------------------------------------------------------------
+# pins (each takes an optional ctypes lib so the mutation test can rerun them)
+# ----------------------------------------------------------------------------------------
+def pin_closed_form(oracle_mod, lib=None):
+    for (H, W, N, seed) in [(8, 8, 4, 0), (5, 7, 3, 1), (6, 3, 2, 2)]:
+        d = _small(H=H, W=W, N=N, channels=2, batch=1, seed=seed)
+        y = _fwd(oracle_mod, d, lib)
+        for ch in range(2):
+            ref = closed_form_map(*_map_args(d, 0, ch))
+            np.testing.assert_allclose(y[0, ch], ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_linsolve(oracle_mod, lib=None):
+    d = _small(H=7, W=9, N=3, channels=2, batch=2, seed=3, random_A=True)
+    y = _fwd(oracle_mod, d, lib)
+    for b in range(2):
+        for ch in range(2):
+            ref = linsolve_map(*_map_args(d, b, ch))
+            np.testing.assert_allclose(y[b, ch], ref, rtol=1e-11, atol=1e-11)
+
+
+def pin_manhattan_constant(oracle_mod, lib=None):
+    """Constant delta and A: h[i,j] = sum a^{(i-i')+(j-j')} Bbar x  (pages' printed form)."""
+    d = _small(H=6, W=9, N=2, channels=1, batch=1, seed=4)
+    d["delta"][:] = np.float32(0.3)
+    y = _fwd(oracle_mod, d, lib)
+    x, dl, A, B, C, D = _map_args(d, 0, 0)
+    H, W = x.shape
+    ii, jj = np.meshgrid(np.arange(H), np.arange(W), indexing="ij")
+    ref = D * x
+    for n in range(A.shape[0]):
+        a = np.exp(dl[0, 0] * A[n])        # the stored fp32 value of delta
+        u = dl * B[n] * x
+        h = np.zeros((H, W))
+        for i in range(H):
+            for j in range(W):
+                m = (ii <= i) & (jj <= j)
+                h[i, j] = np.sum(a ** ((i - ii[m]) + (j - jj[m])) * u[m])
+        ref = ref + C[n] * h
+    np.testing.assert_allclose(y[0, 0], ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_golden_3x3(oracle_mod, lib=None):
+    g = json.load(open(os.path.join(GOLDEN, "manhattan_3x3.json")))
+    H, W = g["H"], g["W"]
+    si, sj = (v - 1 for v in g["source_1based"])
+    ti, tj = (v - 1 for v in g["target_1based"])
+    dval, aval = 0.25, -1.5
+    x = np.zeros((1, 1, H, W), np.float32)
+    x[0, 0, si, sj] = 1.0
+    delta = np.full((1, 1, H, W), dval, np.float32)
+    A = np.array([[aval]], np.float32)
+    B = np.ones((1, 1, 1, H, W), np.float32)
+    C = np.zeros((1, 1, 1, H, W), np.float32)
+    C[0, 0, 0, ti, tj] = 1.0
+    y = oracle_mod.scan2d_fwd(x, delta, A, B, C, None, 1, lib=lib)
+    abar = np.exp(np.float64(np.float32(dval)) * np.float64(np.float32(aval)))
+    bbar_x = np.float64(np.float32(dval))
+    assert y[0, 0, ti, tj] == pytest.approx(abar ** g["power_2d"] * bbar_x, rel=1e-13)
+    # the flattened 1D sequence of the same map decays with the sequence distance
+    flat = recurrence_1d(np.full(H * W, abar), np.eye(H * W)[si * W + sj] * bbar_x)
+    assert flat[ti * W + tj] == pytest.approx(abar ** g["power_1d_flattened"] * bbar_x, rel=1e-13)
+    assert g["power_2d"] == (ti - si) + (tj - sj)
+
+
+def pin_1d_reduction(oracle_mod, lib=None):
+    for (H, W) in [(1, 13), (11, 1)]:
+        d = _small(H=H, W=W, N=3, channels=2, batch=1, seed=5, random_A=True)
+        y = _fwd(oracle_mod, d, lib)
+        for ch in range(2):
+            x, dl, A, B, C, D = _map_args(d, 0, ch)
+            ref = D * x.ravel()
+            for n in range(A.shape[0]):
+                h = recurrence_1d(np.exp(dl * A[n]).ravel(), (dl * B[n] * x).ravel())
+                ref = ref + C[n].ravel() * h
+            np.testing.assert_allclose(y[0, ch].ravel(), ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_linearity_and_special(oracle_mod, lib=None):
+    d = _small(H=5, W=6, N=3, channels=3, batch=2, seed=6)
+    y1 = _fwd(oracle_mod, d, lib)
+    Dx = d["Dskip"][None, :, None, None].astype(np.float64) * d["x"].astype(np.float64)
+    d2 = dict(d)
+    d2["x"] = (d["x"] * np.float32(2.0)).astype(np.float32)
+    y2 = _fwd(oracle_mod, d2, lib)
+    np.testing.assert_allclose(y2 - 2 * Dx, 2 * (y1 - Dx), rtol=1e-12, atol=1e-12)
+    # B = 0: only the skip term remains
+    d3 = dict(d)
+    d3["B"] = np.zeros_like(d["B"])
+    np.testing.assert_array_equal(_fwd(oracle_mod, d3, lib), Dx)
+    # C = e_n at one position picks that state's h; compare with the closed form
+    d4 = dict(d)
+    d4["C"] = np.zeros_like(d["C"])
+    d4["C"][:, :, 1] = 1.0
+    d4["Dskip"] = None
+    y4 = _fwd(oracle_mod, d4, lib)
+    x, dl, A, B, C, D = _map_args(d4, 1, 2)
+    ref = closed_form_map(x, dl, A[1:2], B[1:2], C[1:2], 0.0)
+    np.testing.assert_allclose(y4[1, 2], ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_orientations(oracle_mod, lib=None):
+    """Four orientations = four top-left scans of the flipped map, flipped back, + D x once."""
+    d = _small(H=5, W=7, N=2, channels=2, batch=1, seed=7, orient_mask=0xF)
+    y = _fwd(oracle_mod, d, lib)
+    ref = d["Dskip"][None, :, None, None].astype(np.float64) * d["x"].astype(np.float64)
+    for k, (fh, fw) in enumerate([(0, 0), (0, 1), (1, 0), (1, 1)]):
+        axes = tuple(ax for ax, f in ((2, fh), (3, fw)) if f)
+        fl = (lambda a: np.flip(a, axes).copy()) if axes else (lambda a: a.copy())
+        flb = (lambda a: np.flip(a, tuple(ax + 1 for ax in axes)).copy()) if axes else (lambda a: a.copy())
+        yk = oracle_mod.scan2d_fwd(fl(d["x"]), fl(d["delta"]), d["A"], flb(d["B"][:, k:k + 1]),
+                                   flb(d["C"][:, k:k + 1]), None, 1)
+        ref = ref + fl(yk)
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+    # and a subset mask uses B_k, C_k in set-bit order
+    d2 = dict(d)
+    d2["B"] = d["B"][:, [1, 3]].copy()
+    d2["C"] = d["C"][:, [1, 3]].copy()
+    y2 = _fwd(oracle_mod, d2, lib, mask=0b1010)
+    d3 = dict(d)
+    d3["B"] = d["B"][:, [1]].copy()
+    d3["C"] = d["C"][:, [1]].copy()
+    d4 = dict(d)
+    d4["B"] = d["B"][:, [3]].copy()
+    d4["C"] = d["C"][:, [3]].copy()
+    Dx = d["Dskip"][None, :, None, None].astype(np.float64) * d["x"].astype(np.float64)
+    ysum = _fwd(oracle_mod, d3, lib, mask=0b0010) + _fwd(oracle_mod, d4, lib, mask=0b1000) - Dx
+    np.testing.assert_allclose(y2, ysum, rtol=1e-12, atol=1e-12)
+
+
+def pin_points_and_maps(oracle_mod, lib=None):
+    d = _small(H=9, W=11, N=3, channels=3, batch=2, seed=8, orient_mask=0b1101)
+    y = _fwd(oracle_mod, d, lib)
+    pts = [(0, 0, 0, 0), (1, 2, 8, 10), (0, 1, 4, 0), (1, 0, 0, 10), (1, 1, 5, 6)]
+    yp = oracle_mod.scan2d_points(d["x"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"], pts,
+                                  d["orient_mask"], lib=lib)
+    np.testing.assert_allclose(yp, [y[p] for p in pts], rtol=1e-13, atol=1e-13)
+    ym = oracle_mod.scan2d_maps(d["x"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"],
+                                [(1, 2), (0, 1)], d["orient_mask"], lib=lib)
+    np.testing.assert_array_equal(ym[0], y[1, 2])
+    np.testing.assert_array_equal(ym[1], y[0, 1])
+
+
+PINS = [pin_closed_form, pin_linsolve, pin_manhattan_constant, pin_golden_3x3,
+        pin_1d_reduction, pin_linearity_and_special, pin_orientations, pin_points_and_maps]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
+def test_pin(oracle_mod, pin):
+    pin(oracle_mod)
+
+
+def test_bf16_inputs_widen_exactly(oracle_mod):
+    d = _small(H=6, W=5, N=3, channels=2, batch=1, seed=9, dtype="bf16", orient_mask=0b0110)
+    y = _fwd(oracle_mod, d)
+    f = dict(d)
+    for k in ("x", "delta", "B", "C"):
+        f[k] = inputs.bf16_bits_to_f32(d[k])
+    np.testing.assert_array_equal(y, _fwd(oracle_mod, f))
+
+
+def test_bf16_rounding_is_nearest_even():
+    v = np.array([1.0, 1.00390625, 1.005859375, -2.5, 3.0e-3], np.float32)
+    bits = inputs.f32_to_bf16_bits(v)
+    back = inputs.bf16_bits_to_f32(bits)
+    # 1 + 2^-8 is a tie between 1 and 1 + 2^-7: even mantissa (1.0) wins
+    assert back[0] == 1.0 and back[1] == 1.0
+    assert back[2] == np.float32(1.0078125)
+    assert back[3] == -2.5
+    assert abs(back[4] - 3.0e-3) <= 3.0e-3 * 2 ** -8
+
+
+def test_oracle_rejects_bad_arguments(oracle_mod):
+    d = _small()
+    with pytest.raises((RuntimeError, ValueError)):
+        _fwd(oracle_mod, d, mask=0)
+    with pytest.raises(RuntimeError):
+        oracle_mod.scan2d_points(d["x"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"],
+                                 [(0, 0, 8, 0)], 1)
+
+
+# ----------------------------------------------------------------------------------------
+# planted mistakes: a copy of the oracle with one plausible error must fail some pin
+# ----------------------------------------------------------------------------------------
+MUTATIONS = {
+    "vertical_without_decay": ("hcol[jj] = abar * hcol[jj] + hh;", "hcol[jj] = hcol[jj] + hh;"),
+    "bbar_without_delta": ("hh = abar * hh + (dl * Bv) * xv;", "hh = abar * hh + Bv * xv;"),
+    "exp_sign": ("exp(dl * An)", "exp(-dl * An)"),
+    "no_skip_term": ("ym[pos] += Dd * load(x, map + pos, is_bf16);", "(void)Dd;"),
+    "flip_w_ignored": ("const int j = flipW ? W - 1 - jj : jj;", "const int j = jj;"),
+    "C_transposed": ("load(p->C, bc + pos, p->is_bf16)",
+                     "load(p->C, bc + ((size_t)j * H + i) % ((size_t)H * W), p->is_bf16)"),
+    "vertical_adds_bbar_again": ("hcol[jj] = abar * hcol[jj] + hh;",
+                                 "hcol[jj] = abar * hcol[jj] + hh + (dl * Bv) * xv;"),
+    "horizontal_carry_not_reset": ("double hh = 0.0;                               /* hh[i, -1] = 0 */",
+                                   "static double hh; if (ii == 0) hh = 0.0;"),
+    "state_index_off_by_one": ("const double An = (double)p->A[(size_t)d * N + n];",
+                               "const double An = (double)p->A[(size_t)d * N + (n + 1) % N];"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(oracle_mod, tmp_path, name):
+    src = open(os.path.join(os.path.dirname(oracle_mod.__file__), "scan2d_oracle.c")).read()
+    old, new = MUTATIONS[name]
+    assert src.count(old) >= 1, f"mutation anchor missing: {old}"
+    mutated = src.replace(old, new)
+    c = tmp_path / "mut.c"
+    so = tmp_path / "libmut.so"
+    c.write_text(mutated)
+    subprocess.check_call(["gcc", "-std=c99", "-O2", "-fPIC", "-shared", "-o", str(so), str(c), "-lm"])
+    lib = oracle_mod.load_library(str(so))
+    caught = []
+    for pin in PINS:
+        try:
+            pin(oracle_mod, lib)
+        except AssertionError:
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught the planted mistake {name}"
