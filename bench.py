@@ -1,0 +1,379 @@
+"""Benchmark of the 2D selective-scan forward on B200: Gelem/s (batch*D*H*W per second) and
+the fraction of the kernel's roofline.  One JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload giga|vision|small|wsi|tiny]
+                    [--impl ours|reference] [--no-cpu-baseline] [--others]
+
+A step is one scan2d_fwd call over one batch of the workload (every step of the path runs
+in it).  N > 1 runs under torchrun, one rank per GPU; the (b, d) maps are independent, so
+each rank runs its own instance of the workload (weak scaling, no collective on the data
+path) and the value is all ranks' elements over the slowest rank's time.
+
+--impl reference times the fp64 oracle (the CPU reference of this path) on the host cores,
+each step a bounded sample of the workload; rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from selective_state_space_scan2d_b200 import inputs  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+SMS = 148
+MUFU_PER_CLK_SM = 16          # ex2 per clock per SM (sm_100 throughput table, confirmed by probe)
+FP32_PER_CLK_SM = 128         # FP32 lanes per clock per SM
+SM_MAX_MHZ = 1965.0
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured", float(p.get("sm_max_mhz", SM_MAX_MHZ))
+    except Exception:
+        return 6650.0, "fallback", SM_MAX_MHZ
+
+
+def roofline_model(w: inputs.Workload):
+    """Algorithmic work per element (batch*D*H*W unit) and the bound at peak rates."""
+    s = 2 if w.dtype == "bf16" else 4
+    sy = s
+    bytes_el = 2 * s + sy + w.K * 2 * w.N * s / w.channels
+    exps_el = w.N                                   # Abar once per (position, state)
+    fp32_el = w.N * (1 + 4 * w.K) + 2               # dA mul; per orientation Bbar x, hor, vert, C
+    hbm_gbs, hbm_kind, sm_mhz = _peaks()
+    clk = sm_mhz * 1e6
+    t_hbm = bytes_el / (hbm_gbs * 1e9)
+    t_sfu = exps_el / (SMS * MUFU_PER_CLK_SM * clk)
+    t_fp32 = fp32_el / (SMS * FP32_PER_CLK_SM * clk)
+    bound = max((t_hbm, "hbm"), (t_sfu, "sfu"), (t_fp32, "fp32"))[1]
+    return dict(bytes_el=bytes_el, exps_el=exps_el, fp32_el=fp32_el, t_hbm=t_hbm, t_sfu=t_sfu,
+                t_fp32=t_fp32, bound=bound, hbm_gbs=hbm_gbs, hbm_kind=hbm_kind, sm_mhz=sm_mhz,
+                roof_gelem=1e-9 / max(t_hbm, t_sfu, t_fp32))
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, torch_dev: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(torch_dev).uuid)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001
+            self.nv = None
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        getr = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = getr(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if self.nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+def _to_dev(a, torch, device):
+    if a is None:
+        return None
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+    return torch.from_numpy(a).to(device)
+
+
+def _to_pinned(a, torch):
+    if a is None:
+        return None
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+    return torch.from_numpy(a).pin_memory()
+
+
+def _oracle_sample_rate(w: inputs.Workload, d: dict, budget_s: float):
+    """Time the fp64 oracle on whole (b, d) maps of the workload, as many as fit the budget."""
+    import oracle
+    oracle.build()
+    maps = [(b, c) for b in range(w.batch) for c in range(w.channels)]
+    done, t_used, elems = 0, 0.0, 0
+    t0 = time.perf_counter()
+    while done < len(maps):
+        # one map at a time until the budget is used
+        oracle.scan2d_maps(d["x"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"], [maps[done]],
+                           d["orient_mask"])
+        done += 1
+        elems += w.H * w.W
+        t_used = time.perf_counter() - t0
+        if t_used >= budget_s:
+            break
+    return elems / t_used / 1e9, done, t_used
+
+
+def run_reference(args, w: inputs.Workload):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    d = inputs.make_inputs(w, seed=0)
+    # one step = whole maps of the workload, about 0.5 s of oracle work
+    maps_all = [(b, c) for b in range(w.batch) for c in range(w.channels)]
+    t0 = time.perf_counter()
+    oracle.scan2d_maps(d["x"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"], [maps_all[0]], d["orient_mask"])
+    t_map = max(time.perf_counter() - t0, 1e-6)
+    per_step = max(1, min(len(maps_all), int(0.5 / t_map)))
+    step_maps = [maps_all[i % len(maps_all)] for i in range(per_step)]
+    for _ in range(args.warmup):
+        oracle.scan2d_maps(d["x"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"], step_maps, d["orient_mask"])
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.scan2d_maps(d["x"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"], step_maps, d["orient_mask"])
+    dt = (time.perf_counter() - t0) / args.steps
+    elems = per_step * w.H * w.W
+    value = elems / dt / 1e9
+    sample = f"{per_step} whole (b,d) maps of {w.name} per step ({elems} elements), fp64 C oracle"
+    print(json.dumps({
+        "impl": "reference", "metric": "2D selective-scan fwd Gelem/s (B*D*H*W)", "value": value,
+        "unit": "Gelem/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "channels": w.channels, "N": w.N,
+                   "H": w.H, "W": w.W, "dtype_in": w.dtype, "orientations": w.K},
+        "cpu_baseline": {"value": value, "unit": "Gelem/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "Gelem/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def measure_workload(w, args, torch, scan2d, device, rank, seed, steps, warmup, with_e2e):
+    d = inputs.make_inputs(w, seed=seed)
+    flags = scan2d.flags_for(w.dtype == "bf16", w.orient_mask)
+    plan = scan2d.scan2d_query_plan(w.batch, w.channels, w.H, w.W, w.N, flags)
+    t = {k: _to_dev(d[k], torch, device) for k in ("x", "delta", "A", "B", "C", "Dskip")}
+    set_bytes = sum(v.numel() * v.element_size() for v in t.values() if v is not None)
+    out_dtype = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    y_bytes = w.elements * (2 if w.dtype == "bf16" else 4)
+    set_bytes += y_bytes
+    # rotate through copies of the inputs so that no step finds its data in L2
+    n_sets = max(1, math.ceil(3 * L2_BYTES / set_bytes))
+    sets = [t] + [{k: (v.clone() if v is not None else None) for k, v in t.items()} for _ in range(n_sets - 1)]
+    ys = [torch.empty((w.batch, w.channels, w.H, w.W), dtype=out_dtype, device=device) for _ in range(n_sets)]
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        s = sets[i % n_sets]
+        scan2d.scan2d_fwd(s["x"], s["delta"], s["A"], s["B"], s["C"], s["Dskip"], y=ys[i % n_sets],
+                          flags=flags, stream=stream)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if torch.distributed.is_initialized():
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index) as clk:
+        e0.record(stream)
+        for i in range(steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    if torch.distributed.is_initialized():
+        torch.distributed.barrier()
+    ms = e0.elapsed_time(e1) / steps
+    err = scan2d.scan2d_get_device_error()
+    if err:
+        raise RuntimeError(f"device error {err}: {scan2d.scan2d_strerror(err)}")
+    res = dict(ms=ms, plan=plan, n_sets=n_sets, clocks=clk.summary(), flags=flags, d=d)
+    if with_e2e:
+        res["e2e"] = measure_e2e(w, d, torch, scan2d, device, flags, steps)
+    del sets, ys, t
+    return res
+
+
+def measure_e2e(w, d, torch, scan2d, device, flags, steps):
+    """scan2d_fwd_host on pinned host buffers: H2D of the inputs, the scan, D2H of y."""
+    h = {k: _to_pinned(d[k], torch) for k in ("x", "delta", "A", "B", "C", "Dskip")}
+    out_dtype = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    yh = torch.empty((w.batch, w.channels, w.H, w.W), dtype=out_dtype).pin_memory()
+    nbytes = scan2d.scan2d_host_staging_bytes(w.batch, w.channels, w.H, w.W, w.N, flags)
+    staging = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    n = max(2, min(steps, 10))
+    scan2d.scan2d_fwd_host(h["x"], h["delta"], h["A"], h["B"], h["C"], h["Dskip"], yh, staging, flags, stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        scan2d.scan2d_fwd_host(h["x"], h["delta"], h["A"], h["B"], h["C"], h["Dskip"], yh, staging, flags, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    h2d = sum(v.numel() * v.element_size() for v in h.values() if v is not None)
+    d2h = yh.numel() * yh.element_size()
+    return dict(ms=ms, steps=n, h2d=h2d, d2h=d2h)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="giga", choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--others", action="store_true", help="also time the other workloads (extra key)")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    w = inputs.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+
+    import torch
+    from selective_state_space_scan2d_b200 import scan2d
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+
+    res = measure_workload(w, args, torch, scan2d, device, rank, seed=rank, steps=args.steps,
+                           warmup=args.warmup, with_e2e=True)
+    ms = res["ms"]
+    e2e_ms = res["e2e"]["ms"]
+    if world > 1:
+        t = torch.tensor([ms, e2e_ms], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+    value = world * w.elements / (ms * 1e-3) / 1e9
+    e2e_value = world * w.elements / (e2e_ms * 1e-3) / 1e9
+
+    rm = roofline_model(w)
+    if rm["bound"] == "sfu":
+        achieved = w.elements * rm["exps_el"] / (ms * 1e-3) / 1e9
+        peak = SMS * MUFU_PER_CLK_SM * rm["sm_mhz"] * 1e6 / 1e9
+        unit = "Gex2/s"
+    elif rm["bound"] == "fp32":
+        achieved = w.elements * rm["fp32_el"] / (ms * 1e-3) / 1e9
+        peak = SMS * FP32_PER_CLK_SM * rm["sm_mhz"] * 1e6 / 1e9
+        unit = "Gfp32op/s"
+    else:
+        achieved = w.elements * rm["bytes_el"] / (ms * 1e-3) / 1e9
+        peak = rm["hbm_gbs"]
+        unit = "GB/s"
+    roof = {"bound": "alu" if rm["bound"] != "hbm" else "hbm", "unit_of_bound": rm["bound"],
+            "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+            "traffic": None, "peak_kind": f"nominal {SMS} SMs x {MUFU_PER_CLK_SM if rm['bound']=='sfu' else FP32_PER_CLK_SM}/clk x {rm['sm_mhz']:.0f} MHz (max clock)" if rm["bound"] != "hbm" else f"{rm['hbm_kind']} copy bandwidth",
+            "hbm_achieved_gbs": w.elements * rm["bytes_el"] / (ms * 1e-3) / 1e9,
+            "hbm_frac_of_measured": w.elements * rm["bytes_el"] / (ms * 1e-3) / 1e9 / rm["hbm_gbs"],
+            "roofline_gelem_s": rm["roof_gelem"], "frac_of_roofline_gelem": (w.elements / (ms * 1e-3) / 1e9) / rm["roof_gelem"]}
+    clocks = res["clocks"]
+    if clocks.get("sm_mhz"):
+        roof["frac_at_sampled_clock"] = roof["frac"] * (rm["sm_mhz"] / clocks["sm_mhz"]) if rm["bound"] != "hbm" else roof["frac"]
+
+    line = {
+        "metric": "2D selective-scan fwd Gelem/s (B*D*H*W) and % of HBM/SFU roofline",
+        "value": value, "unit": "Gelem/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32" if w.dtype == "f32" else "bf16-in/f32-acc",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "channels": w.channels, "N": w.N,
+                   "H": w.H, "W": w.W, "dtype_in": w.dtype, "orientations": w.K,
+                   "global_batch": w.batch * world, "parallelism": f"replicas x{world}",
+                   "l2": f"inputs rotated over {res['n_sets']} device copies (> 3x L2 per rotation)"},
+        "roofline": roof,
+        "clocks": clocks,
+        "gpu_launches": args.steps * res["plan"]["launches"],
+        "plan": res["plan"],
+        "e2e": {"value": e2e_value, "unit": "Gelem/s", "h2d_bytes_per_step": res["e2e"]["h2d"],
+                "d2h_bytes_per_step": res["e2e"]["d2h"], "steps": res["e2e"]["steps"],
+                "api": "scan2d_fwd_host (pinned host buffers)"},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, nmaps, secs = _oracle_sample_rate(w, res["d"], args.cpu_budget)
+        line["cpu_baseline"] = {"value": rate, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{nmaps} whole (b,d) maps of {w.name} ({nmaps * w.H * w.W} elements) in {secs:.1f} s, fp64 C oracle, 1 thread"}
+    if args.others and world == 1:
+        others = {}
+        for name in ("wsi", "small", "vision", "giga"):
+            if name == w.name:
+                continue
+            ow = inputs.WORKLOADS[name]
+            r = measure_workload(ow, args, torch, scan2d, device, rank, seed=0,
+                                 steps=max(20, args.steps // 4), warmup=args.warmup, with_e2e=False)
+            orm = roofline_model(ow)
+            gel = ow.elements / (r["ms"] * 1e-3) / 1e9
+            others[name] = {"value": gel, "ms_per_step": r["ms"], "bound": orm["bound"],
+                            "roofline_gelem_s": orm["roof_gelem"], "frac": gel / orm["roof_gelem"],
+                            "clocks": r["clocks"], "plan": r["plan"]}
+        line["others"] = others
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

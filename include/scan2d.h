@@ -1,0 +1,148 @@
+/*
+ * scan2d.h -- C ABI of the B200 (sm_100a) 2D selective-scan forward (2DMamba).
+ *
+ * Operation (sources are web pages on 2DMamba, arXiv 2412.00678):
+ *   "2DMamba 精读：从小白到博士" (juejin.cn), section 四.5 "2DMamba 如何扩展到二维？":
+ *     (1) horizontal scan   hh[i,j] = Abar[i,j] * hh[i,j-1] + Bbar[i,j] * x[i,j]
+ *     (2) vertical scan     h[i,j]  = Abar[i,j] * h[i-1,j]  + hh[i,j]
+ *         output            y[i,j]  = C h[i,j]
+ *   papernotes.org notes on the CVPR 2025 paper, "关键设计": the hardware-aware operator
+ *   keeps the N states on chip and writes only the reduced output, so memory traffic is
+ *   O(L) rather than O(N L).
+ * For every (b, d) map and state n this library computes, with the same Abar in both scans,
+ *   Abar = exp(delta[b,d,i,j] * A[d,n]),   Bbar = delta[b,d,i,j] * B[b,k,n,i,j],
+ *   y[b,d,i,j] = sum_k sum_n C[b,k,n,i,j] * h_k[n,i,j] + Dskip[d] * x[b,d,i,j],
+ * with zero initial states (hh[i,-1] = 0, h[-1,j] = 0).  The discretisation, the initial
+ * states, the skip term and the orientation semantics are not printed on the pages; the
+ * plainest readings are taken (see the design notes shipped with the repository).
+ *
+ * Orientations ("reverse scans" in the papernotes "局限与展望", "四象限" in the juejin
+ * section 七.4): orientation TL scans from the top-left corner; TR from the top-right
+ * (W reversed); BL from the bottom-left (H reversed); BR from the bottom-right.  Each
+ * orientation k has its own B_k, C_k; delta, A and Dskip are shared and Dskip * x is added
+ * once.  K = number of orientation bits set (default TL only, K = 1).
+ *
+ * Layouts: dense, contiguous, row-major with W fastest.
+ *   x, delta, y : (batch, channels, H, W)
+ *   A           : (channels, N)            fp32
+ *   B, C        : (batch, K, N, H, W)      shared by all channels; for K = 1 this is
+ *                                          (batch, N, H, W); orientations in bit order
+ *                                          TL, TR, BL, BR
+ *   Dskip       : (channels)               fp32, may be NULL (then 0)
+ * Element types: fp32 by default; with SCAN2D_BF16, x, delta, B, C and y are bf16 (y fp32
+ * instead with SCAN2D_OUT_F32).  Arithmetic is fp32 throughout.
+ *
+ * Ownership: the caller owns every buffer.  scan2d_fwd never frees or retains a caller
+ * pointer past the call.  It keeps, per (device, stream), a small internal workspace for
+ * cross-block carries (and, for several orientations on maps too large for shared memory
+ * with bf16 output, an fp32 accumulator); it is created with cudaMalloc on first need and
+ * grown on demand, which synchronises that stream once.  Make a first call of each shape
+ * before capturing a stream into a CUDA graph.  Calls on different streams use different
+ * workspaces and may run concurrently.
+ *
+ * Errors: every entry point returns 0 on success or a negative SCAN2D_E_* code, and never
+ * aborts or throws.  Argument errors are detected on the host before anything is launched.
+ * Device-side failures (a bounded wait for a neighbouring block that ran out) are reported
+ * by scan2d_get_device_error() after the work has completed.
+ */
+#ifndef SCAN2D_H
+#define SCAN2D_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- flags ----------------------------------------------------------------------- */
+#define SCAN2D_BF16     0x1u   /* x, delta, B, C (and y) are bf16 instead of fp32      */
+#define SCAN2D_OUT_F32  0x2u   /* with SCAN2D_BF16: y is fp32                          */
+#define SCAN2D_OR_TL    0x10u  /* orientation: from the top-left corner (default)     */
+#define SCAN2D_OR_TR    0x20u  /* from the top-right corner (W reversed)              */
+#define SCAN2D_OR_BL    0x40u  /* from the bottom-left corner (H reversed)            */
+#define SCAN2D_OR_BR    0x80u  /* from the bottom-right corner (H and W reversed)     */
+#define SCAN2D_OR_ALL   0xF0u
+#define SCAN2D_FLAGS_KNOWN 0xF3u
+
+/* ---- limits ---------------------------------------------------------------------- */
+#define SCAN2D_MAX_N    64     /* states per channel                                   */
+
+/* ---- error codes ----------------------------------------------------------------- */
+#define SCAN2D_OK          0
+#define SCAN2D_E_NULL     -1   /* a required pointer is NULL                            */
+#define SCAN2D_E_DIMS     -2   /* batch, channels, H or W < 1, or a size overflows      */
+#define SCAN2D_E_N        -3   /* N < 1 or N > SCAN2D_MAX_N                             */
+#define SCAN2D_E_FLAGS    -4   /* unknown flag bits, or SCAN2D_OUT_F32 without BF16     */
+#define SCAN2D_E_ALIGN    -5   /* a pointer is not aligned to its element size          */
+#define SCAN2D_E_LAUNCH   -6   /* the CUDA runtime rejected a launch or a copy          */
+#define SCAN2D_E_TIMEOUT  -7   /* device: a bounded wait on a neighbouring block gave up */
+#define SCAN2D_E_NOMEM    -8   /* the internal workspace could not be allocated         */
+#define SCAN2D_E_DEVICE   -9   /* no usable CUDA device, or not an sm_100 device        */
+#define SCAN2D_E_STAGING -10   /* scan2d_fwd_host: staging buffer too small             */
+
+/*
+ * scan2d_fwd -- the 2D selective-scan forward on device buffers.
+ *   x, delta, B, C, y : device pointers, element type per flags (see above);
+ *   A, Dskip          : device pointers to fp32 (Dskip may be NULL);
+ *   batch, channels, H, W >= 1;  1 <= N <= SCAN2D_MAX_N;
+ *   flags             : SCAN2D_BF16 | SCAN2D_OUT_F32 | orientation bits;
+ *   stream            : a cudaStream_t (NULL = the legacy default stream).
+ * Asynchronous: returns once the work is enqueued on `stream`.  y must not alias an input.
+ * Returns 0, or SCAN2D_E_NULL / _DIMS / _N / _FLAGS / _ALIGN / _NOMEM / _LAUNCH / _DEVICE.
+ */
+int scan2d_fwd(const void *x, const void *delta, const float *A, const void *B, const void *C,
+               const float *Dskip, void *y, int batch, int channels, int H, int W, int N,
+               unsigned flags, void *stream);
+
+/*
+ * scan2d_query_plan -- how scan2d_fwd would run a call of this shape, without launching
+ * anything or touching a device.  Writes up to n_out (<= SCAN2D_PLAN_FIELDS) values to `out`:
+ *   [0] kernel launches per call        [5] columns per warp strip
+ *   [1] blocks per launch               [6] warps (strips) per chain in a block
+ *   [2] threads per block               [7] 0 one orientation, 1 orientations summed in
+ *   [3] dynamic shared memory bytes         shared memory, 2 one launch per orientation
+ *   [4] blocks per chain (segments)     [8] states per lane   [9] workspace bytes
+ * Returns 0 or the argument-check codes of scan2d_fwd.
+ */
+#define SCAN2D_PLAN_FIELDS 10
+int scan2d_query_plan(int batch, int channels, int H, int W, int N, unsigned flags,
+                      long long *out, int n_out);
+
+/*
+ * scan2d_host_staging_bytes -- device bytes scan2d_fwd_host needs for one call of this
+ * shape (all inputs and the output, each rounded up to 256 bytes).  0 on bad arguments.
+ */
+size_t scan2d_host_staging_bytes(int batch, int channels, int H, int W, int N, unsigned flags);
+
+/*
+ * scan2d_fwd_host -- scan2d_fwd on HOST buffers.  Copies x, delta, A, B, C, Dskip from the
+ * host into `staging` (a device buffer of at least scan2d_host_staging_bytes(...) bytes,
+ * owned by the caller), runs scan2d_fwd there, and copies y back to the host buffer `y`,
+ * all enqueued on `stream` with one cudaMemcpyAsync per tensor.  Asynchronous: host buffers
+ * must stay valid until the stream has completed; use pinned host memory for the copies to
+ * overlap.  Returns the scan2d_fwd codes, or SCAN2D_E_STAGING.
+ */
+int scan2d_fwd_host(const void *x, const void *delta, const float *A, const void *B,
+                    const void *C, const float *Dskip, void *y, void *staging,
+                    size_t staging_bytes, int batch, int channels, int H, int W, int N,
+                    unsigned flags, void *stream);
+
+/*
+ * scan2d_get_device_error -- synchronises `stream`, then returns and clears the first
+ * device-side error recorded on the current device since the last call (0 if none;
+ * SCAN2D_E_TIMEOUT if a bounded inter-block wait gave up, in which case the output of
+ * the affected call is undefined), or SCAN2D_E_LAUNCH if the stream itself reports an error.
+ */
+int scan2d_get_device_error(void *stream);
+
+/* Human-readable text for a SCAN2D_E_* code (static storage, never NULL). */
+const char *scan2d_strerror(int code);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int scan2d_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SCAN2D_H */

@@ -1,0 +1,418 @@
+// scan2d.cu -- C ABI of the 2D selective-scan forward: argument checks, work planning,
+// per-(device, stream) workspace, kernel dispatch.  The arithmetic is in scan2d_kernels.cuh.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "../../include/scan2d.h"
+#include "scan2d_kernels.cuh"
+
+namespace scan2d {
+
+namespace {
+
+constexpr long long kTimeoutNs = 2000000000LL;   // bounded inter-block waits: 2 s
+constexpr size_t kAlign = 256;
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+int popcount4(unsigned v) { return ((v >> 0) & 1) + ((v >> 1) & 1) + ((v >> 2) & 1) + ((v >> 3) & 1); }
+
+struct Shape {
+  int batch, channels, H, W, N, K;
+  bool bf16, out_f32;
+  unsigned orient;             // 4-bit orientation mask
+  size_t in_elem, out_elem;    // bytes per element of x/delta/B/C and of y
+  size_t xy_count, bc_count;   // elements of x (= y) and of B (= C)
+};
+
+int check_shape(int batch, int channels, int H, int W, int N, unsigned flags, Shape* s) {
+  if (flags & ~SCAN2D_FLAGS_KNOWN) return SCAN2D_E_FLAGS;
+  if ((flags & SCAN2D_OUT_F32) && !(flags & SCAN2D_BF16)) return SCAN2D_E_FLAGS;
+  if (batch < 1 || channels < 1 || H < 1 || W < 1) return SCAN2D_E_DIMS;
+  if (N < 1 || N > SCAN2D_MAX_N) return SCAN2D_E_N;
+  const unsigned long long hw = static_cast<unsigned long long>(H) * W;
+  if (hw > (1ull << 31) - 1) return SCAN2D_E_DIMS;                 // in-map offsets are int
+  unsigned orient = (flags >> 4) & 0xFu;
+  if (orient == 0) orient = 1;                                       // default: top-left
+  const int K = popcount4(orient);
+  const unsigned long long xy = static_cast<unsigned long long>(batch) * channels * hw;
+  const unsigned long long bc = static_cast<unsigned long long>(batch) * K * N * hw;
+  if (xy > (1ull << 40) || bc > (1ull << 40)) return SCAN2D_E_DIMS;
+  s->batch = batch; s->channels = channels; s->H = H; s->W = W; s->N = N; s->K = K;
+  s->bf16 = (flags & SCAN2D_BF16) != 0;
+  s->out_f32 = !s->bf16 || (flags & SCAN2D_OUT_F32) != 0;
+  s->orient = orient;
+  s->in_elem = s->bf16 ? 2 : 4;
+  s->out_elem = s->out_f32 ? 4 : 2;
+  s->xy_count = static_cast<size_t>(xy);
+  s->bc_count = static_cast<size_t>(bc);
+  return SCAN2D_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ---- kernel table ----------------------------------------------------------------------
+using KernelFn = void (*)(const Params);
+
+template <typename Tin, typename Tout>
+KernelFn pick_ng(int ng) {
+  switch (ng) {
+    case 1: return scan2d_strip_kernel<Tin, Tout, 1, 16>;
+    case 2: return scan2d_strip_kernel<Tin, Tout, 2, 16>;
+    case 4: return scan2d_strip_kernel<Tin, Tout, 4, 16>;
+    case 8: return scan2d_strip_kernel<Tin, Tout, 8, 8>;
+    default: return scan2d_strip_kernel<Tin, Tout, 16, 4>;
+  }
+}
+
+int states_per_lane(int N) {
+  int ng = 1;
+  while (ng * kStateLanes < N) ng *= 2;
+  return ng;                       // 1, 2, 4, 8 or 16 for N <= 64
+}
+
+int cmax_for(int ng) { return ng <= 4 ? 16 : (ng == 8 ? 8 : 4); }
+
+KernelFn pick_kernel(const Shape& s, int ng) {
+  if (!s.bf16) return pick_ng<float, float>(ng);
+  if (s.out_f32) return pick_ng<uint16_t, float>(ng);
+  return pick_ng<uint16_t, uint16_t>(ng);
+}
+
+// ---- work plan ---------------------------------------------------------------------------
+struct Plan {
+  int ng, cols, wpc, nseg, chains_per_block, n_cgroups, n_chains, warps;
+  size_t carry_smem;
+};
+
+Plan make_plan(const Shape& s) {
+  Plan pl{};
+  pl.ng = states_per_lane(s.N);
+  const int cmax = cmax_for(pl.ng);
+  pl.n_cgroups = (s.channels + kChanPerWarp - 1) / kChanPerWarp;
+  pl.n_chains = s.batch * pl.n_cgroups;
+  const int strips = (s.W + cmax - 1) / cmax;
+  if (strips == 1) {
+    pl.cols = s.W;
+    pl.wpc = 1;
+    pl.nseg = 1;
+    pl.chains_per_block = 4;
+  } else {
+    pl.cols = (s.W + strips - 1) / strips;                   // balanced strips
+    const int nstrips = (s.W + pl.cols - 1) / pl.cols;
+    pl.wpc = nstrips < kMaxWarps ? nstrips : kMaxWarps;
+    pl.nseg = (nstrips + pl.wpc - 1) / pl.wpc;
+    pl.chains_per_block = 1;
+  }
+  pl.warps = pl.wpc * pl.chains_per_block;
+  pl.carry_smem = pl.wpc > 1 ? sizeof(float) * 2 * kMaxWarps * 32 * pl.ng : 0;
+  return pl;
+}
+
+// ---- per-(device, stream) workspace --------------------------------------------------------
+struct Workspace {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+  unsigned long long gen = 0;
+};
+
+std::mutex g_mu;
+std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+
+// Returns a zero-initialised (at creation) workspace of at least `bytes` bytes, or null.
+Workspace* get_workspace(int dev, cudaStream_t st, size_t bytes) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace& ws = g_ws[std::make_pair(dev, st)];
+  if (ws.bytes < bytes) {
+    if (ws.ptr != nullptr) {
+      if (cudaStreamSynchronize(st) != cudaSuccess) return nullptr;
+      cudaFree(ws.ptr);
+      ws.ptr = nullptr;
+      ws.bytes = 0;
+    }
+    size_t want = round_up(bytes, 1 << 20);
+    if (cudaMalloc(&ws.ptr, want) != cudaSuccess) {
+      cudaGetLastError();
+      ws.ptr = nullptr;
+      return nullptr;
+    }
+    if (cudaMemsetAsync(ws.ptr, 0, want, st) != cudaSuccess) {
+      cudaFree(ws.ptr);
+      ws.ptr = nullptr;
+      return nullptr;
+    }
+    ws.bytes = want;
+    ws.gen = 0;
+  }
+  return &ws;
+}
+
+int launch(KernelFn fn, const Plan& pl, Params prm, size_t smem, int grid, cudaStream_t st) {
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess) {
+      cudaGetLastError();
+      return SCAN2D_E_LAUNCH;
+    }
+  }
+  fn<<<grid, pl.warps * 32, smem, st>>>(prm);
+  if (cudaGetLastError() != cudaSuccess) return SCAN2D_E_LAUNCH;
+  return SCAN2D_OK;
+}
+
+int device_ok(int* dev, int* nsm) {
+  if (cudaGetDevice(dev) != cudaSuccess) { cudaGetLastError(); return SCAN2D_E_DEVICE; }
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(nsm, cudaDevAttrMultiProcessorCount, *dev) != cudaSuccess) {
+    cudaGetLastError();
+    return SCAN2D_E_DEVICE;
+  }
+  if (major != 10) return SCAN2D_E_DEVICE;
+  return SCAN2D_OK;
+}
+
+}  // namespace
+
+// Everything a call of this shape launches, without touching memory.
+struct CallPlan {
+  Plan pl;
+  KernelFn fn;
+  int codes[4], nk;
+  bool smem_multi, global_multi, need_yacc_ws, need_ws;
+  int yacc_stride, grid, launches;
+  size_t smem, off_ctrl, off_flags, off_acks, off_carry, off_yacc, ws_bytes;
+};
+
+CallPlan plan_call(const Shape& s) {
+  CallPlan cp{};
+  cp.pl = make_plan(s);
+  const Plan& pl = cp.pl;
+  cp.fn = pick_kernel(s, pl.ng);
+  cp.nk = 0;
+  for (int o = 0; o < 4; ++o)
+    if (s.orient & (1u << o)) cp.codes[cp.nk++] = o;
+  const size_t HW = static_cast<size_t>(s.H) * s.W;
+  size_t yacc_smem = ~size_t(0);
+  cp.yacc_stride = 0;
+  if (HW <= (1u << 20)) {
+    cp.yacc_stride = static_cast<int>(round_up(HW, 32) + 4);          // +4: spread the banks
+    yacc_smem = sizeof(float) * static_cast<size_t>(pl.chains_per_block) * kChanPerWarp * cp.yacc_stride;
+  }
+  cp.smem_multi = s.K > 1 && pl.nseg == 1 && yacc_smem != ~size_t(0) && pl.carry_smem + yacc_smem <= 200 * 1024;
+  cp.global_multi = s.K > 1 && !cp.smem_multi;
+  cp.need_yacc_ws = cp.global_multi && !s.out_f32;
+  const size_t items = static_cast<size_t>(pl.n_chains) * pl.nseg;
+  cp.off_ctrl = 0;
+  cp.off_flags = kAlign;
+  cp.off_acks = cp.off_flags + round_up(items * 8, kAlign);
+  cp.off_carry = cp.off_acks + round_up(items * 8, kAlign);
+  cp.off_yacc = cp.off_carry + round_up(items * kRing * 32 * pl.ng * sizeof(float), kAlign);
+  cp.ws_bytes = cp.off_yacc + (cp.need_yacc_ws ? s.xy_count * sizeof(float) : 0);
+  cp.need_ws = pl.nseg > 1 || cp.need_yacc_ws;
+  if (!cp.need_ws) cp.ws_bytes = 0;
+  cp.grid = pl.nseg > 1 ? pl.n_chains * pl.nseg
+                        : (pl.n_chains + pl.chains_per_block - 1) / pl.chains_per_block;
+  cp.smem = pl.carry_smem + (cp.smem_multi ? yacc_smem : 0);
+  cp.launches = cp.global_multi ? cp.nk : 1;
+  return cp;
+}
+
+int forward(const void* x, const void* delta, const float* A, const void* B, const void* C,
+            const float* Dskip, void* y, int batch, int channels, int H, int W, int N,
+            unsigned flags, cudaStream_t st) {
+  Shape s;
+  int rc = check_shape(batch, channels, H, W, N, flags, &s);
+  if (rc) return rc;
+  if (!x || !delta || !A || !B || !C || !y) return SCAN2D_E_NULL;
+  if (!aligned(x, s.in_elem) || !aligned(delta, s.in_elem) || !aligned(B, s.in_elem) ||
+      !aligned(C, s.in_elem) || !aligned(A, 4) || !aligned(Dskip, 4) || !aligned(y, s.out_elem))
+    return SCAN2D_E_ALIGN;
+  int dev = 0, nsm = 0;
+  rc = device_ok(&dev, &nsm);
+  if (rc) return rc;
+
+  const CallPlan cp = plan_call(s);
+  const Plan& pl = cp.pl;
+
+  Params prm;
+  std::memset(&prm, 0, sizeof prm);
+  prm.x = x; prm.delta = delta; prm.A = A; prm.B = B; prm.C = C; prm.Dskip = Dskip; prm.y = y;
+  prm.batch = batch; prm.channels = channels; prm.H = H; prm.W = W; prm.N = N; prm.K = s.K;
+  prm.n_cgroups = pl.n_cgroups; prm.n_chains = pl.n_chains;
+  prm.cols_per_warp = pl.cols; prm.wpc = pl.wpc; prm.chains_per_block = pl.chains_per_block;
+  prm.nseg = pl.nseg;
+  prm.timeout_ns = kTimeoutNs;
+  prm.yacc_stride = cp.yacc_stride;
+
+  Workspace* ws = nullptr;
+  if (cp.need_ws) {
+    if (pl.nseg > 1) {
+      // a chain's blocks must be able to be resident together (producer back-pressure)
+      int per_sm = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, cp.fn, pl.warps * 32, pl.carry_smem) != cudaSuccess) {
+        cudaGetLastError();
+        return SCAN2D_E_LAUNCH;
+      }
+      if (static_cast<long long>(per_sm) * nsm < pl.nseg) return SCAN2D_E_DIMS;
+    }
+    ws = get_workspace(dev, st, cp.ws_bytes);
+    if (!ws) return SCAN2D_E_NOMEM;
+    char* base = static_cast<char*>(ws->ptr);
+    prm.ctrl = reinterpret_cast<unsigned long long*>(base + cp.off_ctrl);
+    prm.flags = reinterpret_cast<unsigned long long*>(base + cp.off_flags);
+    prm.acks = reinterpret_cast<unsigned long long*>(base + cp.off_acks);
+    prm.carry = reinterpret_cast<float*>(base + cp.off_carry);
+    if (cp.need_yacc_ws) prm.yacc = reinterpret_cast<float*>(base + cp.off_yacc);
+  }
+  if (cp.global_multi && s.out_f32) prm.yacc = static_cast<float*>(y);
+
+  auto next_gen = [&]() -> unsigned long long {
+    if (!ws) return 1ull;
+    std::lock_guard<std::mutex> lk(g_mu);
+    return ++ws->gen;
+  };
+
+  if (!cp.global_multi) {
+    prm.mode = cp.smem_multi ? kSmemMulti : kSingle;
+    prm.orient_count = cp.smem_multi ? cp.nk : 1;
+    for (int k = 0; k < prm.orient_count; ++k) { prm.orient_code[k] = cp.codes[k]; prm.orient_k[k] = k; }
+    prm.gen = next_gen();
+    return launch(cp.fn, pl, prm, cp.smem, cp.grid, st);
+  }
+  for (int k = 0; k < cp.nk; ++k) {
+    prm.mode = k == 0 ? kGlobalFirst : (k == cp.nk - 1 ? kGlobalLast : kGlobalMid);
+    prm.orient_count = 1;
+    prm.orient_code[0] = cp.codes[k];
+    prm.orient_k[0] = k;
+    prm.gen = next_gen();
+    rc = launch(cp.fn, pl, prm, cp.smem, cp.grid, st);
+    if (rc) return rc;
+  }
+  return SCAN2D_OK;
+}
+
+}  // namespace scan2d
+
+// ---- C ABI ---------------------------------------------------------------------------------
+extern "C" {
+
+int scan2d_fwd(const void* x, const void* delta, const float* A, const void* B, const void* C,
+               const float* Dskip, void* y, int batch, int channels, int H, int W, int N,
+               unsigned flags, void* stream) {
+  return scan2d::forward(x, delta, A, B, C, Dskip, y, batch, channels, H, W, N, flags,
+                         static_cast<cudaStream_t>(stream));
+}
+
+int scan2d_query_plan(int batch, int channels, int H, int W, int N, unsigned flags,
+                      long long* out, int n_out) {
+  scan2d::Shape s;
+  const int rc = scan2d::check_shape(batch, channels, H, W, N, flags, &s);
+  if (rc) return rc;
+  if (!out) return SCAN2D_E_NULL;
+  const scan2d::CallPlan cp = scan2d::plan_call(s);
+  const long long v[SCAN2D_PLAN_FIELDS] = {
+      cp.launches, cp.grid, cp.pl.warps * 32, static_cast<long long>(cp.smem), cp.pl.nseg,
+      cp.pl.cols, cp.pl.wpc, cp.smem_multi ? 1 : (cp.global_multi ? 2 : 0), cp.pl.ng,
+      static_cast<long long>(cp.ws_bytes)};
+  for (int k = 0; k < n_out && k < SCAN2D_PLAN_FIELDS; ++k) out[k] = v[k];
+  return SCAN2D_OK;
+}
+
+size_t scan2d_host_staging_bytes(int batch, int channels, int H, int W, int N, unsigned flags) {
+  scan2d::Shape s;
+  if (scan2d::check_shape(batch, channels, H, W, N, flags, &s)) return 0;
+  const size_t a = 256;
+  auto r = [&](size_t v) { return (v + a - 1) / a * a; };
+  return 2 * r(s.xy_count * s.in_elem) + r(static_cast<size_t>(channels) * N * 4) +
+         2 * r(s.bc_count * s.in_elem) + r(static_cast<size_t>(channels) * 4) + r(s.xy_count * s.out_elem);
+}
+
+int scan2d_fwd_host(const void* x, const void* delta, const float* A, const void* B,
+                    const void* C, const float* Dskip, void* y, void* staging,
+                    size_t staging_bytes, int batch, int channels, int H, int W, int N,
+                    unsigned flags, void* stream) {
+  scan2d::Shape s;
+  int rc = scan2d::check_shape(batch, channels, H, W, N, flags, &s);
+  if (rc) return rc;
+  if (!x || !delta || !A || !B || !C || !y || !staging) return SCAN2D_E_NULL;
+  const size_t need = scan2d_host_staging_bytes(batch, channels, H, W, N, flags);
+  if (staging_bytes < need) return SCAN2D_E_STAGING;
+  if (reinterpret_cast<uintptr_t>(staging) % 256) return SCAN2D_E_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t a = 256;
+  auto r = [&](size_t v) { return (v + a - 1) / a * a; };
+  char* p = static_cast<char*>(staging);
+  const size_t bx = s.xy_count * s.in_elem, bA = static_cast<size_t>(channels) * N * 4;
+  const size_t bB = s.bc_count * s.in_elem, bD = static_cast<size_t>(channels) * 4;
+  const size_t by = s.xy_count * s.out_elem;
+  char* dx = p;            p += r(bx);
+  char* dd = p;            p += r(bx);
+  char* dA = p;            p += r(bA);
+  char* dB = p;            p += r(bB);
+  char* dC = p;            p += r(bB);
+  char* dD = p;            p += r(bD);
+  char* dy = p;
+  const cudaMemcpyKind h2d = cudaMemcpyHostToDevice;
+  if (cudaMemcpyAsync(dx, x, bx, h2d, st) != cudaSuccess ||
+      cudaMemcpyAsync(dd, delta, bx, h2d, st) != cudaSuccess ||
+      cudaMemcpyAsync(dA, A, bA, h2d, st) != cudaSuccess ||
+      cudaMemcpyAsync(dB, B, bB, h2d, st) != cudaSuccess ||
+      cudaMemcpyAsync(dC, C, bB, h2d, st) != cudaSuccess ||
+      (Dskip && cudaMemcpyAsync(dD, Dskip, bD, h2d, st) != cudaSuccess)) {
+    cudaGetLastError();
+    return SCAN2D_E_LAUNCH;
+  }
+  rc = scan2d::forward(dx, dd, reinterpret_cast<float*>(dA), dB, dC,
+                       Dskip ? reinterpret_cast<float*>(dD) : nullptr, dy, batch, channels, H, W,
+                       N, flags, st);
+  if (rc) return rc;
+  if (cudaMemcpyAsync(y, dy, by, cudaMemcpyDeviceToHost, st) != cudaSuccess) {
+    cudaGetLastError();
+    return SCAN2D_E_LAUNCH;
+  }
+  return SCAN2D_OK;
+}
+
+int scan2d_get_device_error(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) {
+    cudaGetLastError();
+    return SCAN2D_E_LAUNCH;
+  }
+  int e = 0;
+  if (cudaMemcpyFromSymbol(&e, scan2d::g_device_error, sizeof e) != cudaSuccess) {
+    cudaGetLastError();
+    return SCAN2D_E_LAUNCH;
+  }
+  if (e != 0) {
+    const int zero = 0;
+    cudaMemcpyToSymbol(scan2d::g_device_error, &zero, sizeof zero);
+  }
+  return e;
+}
+
+const char* scan2d_strerror(int code) {
+  switch (code) {
+    case SCAN2D_OK: return "ok";
+    case SCAN2D_E_NULL: return "a required pointer is NULL";
+    case SCAN2D_E_DIMS: return "invalid or too large batch/channels/H/W";
+    case SCAN2D_E_N: return "N out of range (1..SCAN2D_MAX_N)";
+    case SCAN2D_E_FLAGS: return "unknown or inconsistent flags";
+    case SCAN2D_E_ALIGN: return "a pointer is not aligned to its element size";
+    case SCAN2D_E_LAUNCH: return "the CUDA runtime rejected a launch or copy";
+    case SCAN2D_E_TIMEOUT: return "device: a bounded wait on a neighbouring block timed out";
+    case SCAN2D_E_NOMEM: return "workspace allocation failed";
+    case SCAN2D_E_DEVICE: return "no usable sm_100 CUDA device";
+    case SCAN2D_E_STAGING: return "staging buffer too small";
+    default: return "unknown error";
+  }
+}
+
+int scan2d_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,187 @@
+"""ctypes binding of the C ABI in include/scan2d.h (libscan2d_b200.so, built in-tree).
+
+Argument marshalling only: every step of the scan runs in the CUDA library.  There is no
+CPU path; importing this module without the built library raises ImportError.
+
+    y = scan2d_fwd(x, delta, A, B, C, Dskip)          # torch CUDA tensors, y allocated
+    scan2d_fwd(x, delta, A, B, C, Dskip, y=y)         # into a caller-provided y
+
+Tensor layouts (contiguous): x, delta (batch, D, H, W) fp32 or bf16; A (D, N) fp32;
+B, C (batch, K, N, H, W) or (batch, N, H, W) for K = 1, dtype of x; Dskip (D,) fp32 or None.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libscan2d_b200.so")
+
+if not os.path.exists(lib_path):
+    raise ImportError(
+        f"{lib_path} is missing: build it with `python -m selective_state_space_scan2d_b200.build` "
+        "(the 2D scan has no CPU fallback)")
+
+_lib = ctypes.CDLL(lib_path)
+
+_vp, _i, _u, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_size_t
+_lib.scan2d_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _u, _vp]
+_lib.scan2d_fwd.restype = _i
+_lib.scan2d_query_plan.argtypes = [_i, _i, _i, _i, _i, _u, ctypes.POINTER(ctypes.c_longlong), _i]
+_lib.scan2d_query_plan.restype = _i
+_lib.scan2d_host_staging_bytes.argtypes = [_i, _i, _i, _i, _i, _u]
+_lib.scan2d_host_staging_bytes.restype = _sz
+_lib.scan2d_fwd_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i, _i, _i, _i, _i, _u, _vp]
+_lib.scan2d_fwd_host.restype = _i
+_lib.scan2d_get_device_error.argtypes = [_vp]
+_lib.scan2d_get_device_error.restype = _i
+_lib.scan2d_strerror.argtypes = [_i]
+_lib.scan2d_strerror.restype = ctypes.c_char_p
+_lib.scan2d_version.argtypes = []
+_lib.scan2d_version.restype = _i
+
+# flags (include/scan2d.h)
+SCAN2D_BF16 = 0x1
+SCAN2D_OUT_F32 = 0x2
+SCAN2D_OR_TL = 0x10
+SCAN2D_OR_TR = 0x20
+SCAN2D_OR_BL = 0x40
+SCAN2D_OR_BR = 0x80
+
+
+class Scan2dError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {scan2d_strerror(code)} (code {code})")
+
+
+def scan2d_strerror(code: int) -> str:
+    return _lib.scan2d_strerror(int(code)).decode()
+
+
+def scan2d_version() -> int:
+    return int(_lib.scan2d_version())
+
+
+def flags_for(bf16: bool, orient_mask: int = 1, out_f32: bool = False) -> int:
+    """Flag word for an element type and a 4-bit orientation mask (bit0 TL .. bit3 BR)."""
+    f = (SCAN2D_BF16 if bf16 else 0) | ((orient_mask & 0xF) << 4)
+    if out_f32:
+        f |= SCAN2D_OUT_F32
+    return f
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_handle(stream):
+    if stream is None:
+        return _torch().cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _dims(x, B, A):
+    batch, D, H, W = x.shape
+    K = B.shape[1] if B.dim() == 5 else 1
+    N = A.shape[1]
+    return batch, D, H, W, N, K
+
+
+def _check(x, delta, A, B, C, Dskip, device_kind):
+    torch = _torch()
+    for name, t in (("x", x), ("delta", delta), ("A", A), ("B", B), ("C", C), ("Dskip", Dskip)):
+        if t is None:
+            if name != "Dskip":
+                raise ValueError(f"{name} is required")
+            continue
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if device_kind == "cuda" and not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if device_kind == "cpu" and t.is_cuda:
+            raise ValueError(f"{name} must be a host tensor")
+    if x.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("x must be float32 or bfloat16")
+    for name, t in (("delta", delta), ("B", B), ("C", C)):
+        if t.dtype != x.dtype:
+            raise TypeError(f"{name} must have the dtype of x")
+    if A.dtype != torch.float32 or (Dskip is not None and Dskip.dtype != torch.float32):
+        raise TypeError("A and Dskip must be float32")
+
+
+def scan2d_fwd(x, delta, A, B, C, Dskip=None, y=None, flags=None, stream=None):
+    """The 2D selective-scan forward on CUDA tensors (asynchronous on `stream`).
+
+    flags defaults to the element type of x and K = B.shape[1] orientations
+    (TL; TL+TR; TL+TR+BL; all four).  Returns y."""
+    torch = _torch()
+    _check(x, delta, A, B, C, Dskip, "cuda")
+    batch, D, H, W, N, K = _dims(x, B, A)
+    if flags is None:
+        flags = flags_for(x.dtype == torch.bfloat16, (1 << K) - 1)
+    out_dtype = torch.float32 if (x.dtype == torch.float32 or flags & SCAN2D_OUT_F32) else torch.bfloat16
+    if y is None:
+        y = torch.empty((batch, D, H, W), dtype=out_dtype, device=x.device)
+    elif y.dtype != out_dtype or tuple(y.shape) != (batch, D, H, W) or not y.is_contiguous():
+        raise ValueError("y has the wrong dtype, shape or layout")
+    rc = _lib.scan2d_fwd(_ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(Dskip), _ptr(y),
+                         batch, D, H, W, N, flags, _stream_handle(stream))
+    if rc:
+        raise Scan2dError(rc, "scan2d_fwd")
+    return y
+
+
+PLAN_FIELDS = ("launches", "grid", "threads", "smem", "nseg", "cols", "wpc", "mode", "ng",
+               "workspace")
+
+
+def scan2d_query_plan(batch, channels, H, W, N, flags) -> dict:
+    """How scan2d_fwd runs a call of this shape (no device needed)."""
+    out = (ctypes.c_longlong * len(PLAN_FIELDS))()
+    rc = _lib.scan2d_query_plan(batch, channels, H, W, N, flags, out, len(PLAN_FIELDS))
+    if rc:
+        raise Scan2dError(rc, "scan2d_query_plan")
+    return dict(zip(PLAN_FIELDS, (int(v) for v in out)))
+
+
+def scan2d_host_staging_bytes(batch, channels, H, W, N, flags) -> int:
+    return int(_lib.scan2d_host_staging_bytes(batch, channels, H, W, N, flags))
+
+
+def scan2d_fwd_host(x, delta, A, B, C, Dskip, y, staging, flags=None, stream=None):
+    """The forward on HOST tensors (pinned for overlap) through a caller-provided device
+    staging buffer (a uint8 CUDA tensor of scan2d_host_staging_bytes(...) bytes).
+    Asynchronous on `stream`; y (host) is valid once the stream has completed."""
+    torch = _torch()
+    _check(x, delta, A, B, C, Dskip, "cpu")
+    batch, D, H, W, N, K = _dims(x, B, A)
+    if flags is None:
+        flags = flags_for(x.dtype == torch.bfloat16, (1 << K) - 1)
+    rc = _lib.scan2d_fwd_host(_ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(Dskip),
+                              _ptr(y), _ptr(staging), staging.numel() * staging.element_size(),
+                              batch, D, H, W, N, flags, _stream_handle(stream))
+    if rc:
+        raise Scan2dError(rc, "scan2d_fwd_host")
+    return y
+
+
+def scan2d_get_device_error(stream=None) -> int:
+    """Synchronise `stream`; return and clear the device's first recorded error (0 = none)."""
+    return int(_lib.scan2d_get_device_error(_stream_handle(stream)))
+
+
+def raw():
+    """The ctypes library handle, for calls with plain integer pointers."""
+    return _lib

@@ -1,0 +1,127 @@
+"""C-ABI library: builds, loads, exports every function include/scan2d.h declares, and rejects
+bad arguments on the host before touching a device.  No compute calls (no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "scan2d.h")
+
+
+def _header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(scan2d_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def _header_macros():
+    text = open(HEADER).read()
+    return {m.group(1): int(m.group(2), 0)
+            for m in re.finditer(r"#define\s+(SCAN2D_\w+)\s+(-?(?:0x[0-9a-fA-F]+|\d+))u?", text)}
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from selective_state_space_scan2d_b200 import build
+    build.build()
+    from selective_state_space_scan2d_b200 import scan2d
+    return scan2d
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = _header_functions()
+    assert {"scan2d_fwd", "scan2d_fwd_host", "scan2d_get_device_error", "scan2d_strerror",
+            "scan2d_version", "scan2d_host_staging_bytes"} <= set(declared)
+    out = subprocess.run(["nm", "-D", "--defined-only", lib.lib_path], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s+(scan2d_\w+)$", out, flags=re.M))
+    missing = [n for n in declared if n not in exported]
+    assert not missing, f"declared but not exported: {missing}"
+    raw = ctypes.CDLL(lib.lib_path)
+    for n in declared:
+        assert getattr(raw, n) is not None
+
+
+def test_binding_constants_match_header(lib):
+    m = _header_macros()
+    for name in ("SCAN2D_BF16", "SCAN2D_OUT_F32", "SCAN2D_OR_TL", "SCAN2D_OR_TR",
+                 "SCAN2D_OR_BL", "SCAN2D_OR_BR"):
+        assert getattr(lib, name) == m[name], name
+    assert lib.flags_for(True, 0xF, out_f32=True) == (m["SCAN2D_BF16"] | m["SCAN2D_OUT_F32"] | m["SCAN2D_OR_ALL"])
+
+
+def test_version_and_strerror(lib):
+    assert lib.scan2d_version() >= 100
+    m = _header_macros()
+    codes = [v for k, v in m.items() if k.startswith("SCAN2D_E_")]
+    texts = {lib.scan2d_strerror(c) for c in codes}
+    assert len(texts) == len(codes), "every error code has its own text"
+    assert lib.scan2d_strerror(12345) == "unknown error"
+
+
+# fake, 256-byte aligned "device" addresses: the host checks reject the call before any use
+P = 1 << 20
+
+
+@pytest.mark.parametrize("args,code", [
+    # (batch, channels, H, W, N, flags), expected error
+    ((0, 4, 8, 8, 4, 0x10), "SCAN2D_E_DIMS"),
+    ((1, 0, 8, 8, 4, 0x10), "SCAN2D_E_DIMS"),
+    ((1, 4, 0, 8, 4, 0x10), "SCAN2D_E_DIMS"),
+    ((1, 4, 8, -3, 4, 0x10), "SCAN2D_E_DIMS"),
+    ((1, 4, 65536, 65536, 4, 0x10), "SCAN2D_E_DIMS"),
+    ((1, 4, 8, 8, 0, 0x10), "SCAN2D_E_N"),
+    ((1, 4, 8, 8, 65, 0x10), "SCAN2D_E_N"),
+    ((1, 4, 8, 8, 4, 0x100), "SCAN2D_E_FLAGS"),
+    ((1, 4, 8, 8, 4, 0x2), "SCAN2D_E_FLAGS"),        # OUT_F32 without BF16
+    ((1, 4, 8, 8, 4, 0x4), "SCAN2D_E_FLAGS"),        # reserved bit
+])
+def test_host_rejects_bad_shapes(lib, args, code):
+    m = _header_macros()
+    rc = lib.raw().scan2d_fwd(P, P, P, P, P, None, P, *args, None)
+    assert rc == m[code]
+
+
+def test_host_rejects_null_and_misaligned(lib):
+    m = _header_macros()
+    r = lib.raw()
+    dims = (1, 4, 8, 8, 4)
+    for k in range(7):
+        if k == 5:
+            continue                                   # Dskip may be NULL
+        ptrs = [P] * 7
+        ptrs[k] = None
+        assert r.scan2d_fwd(*ptrs, *dims, 0x10, None) == m["SCAN2D_E_NULL"]
+    assert r.scan2d_fwd(P + 2, P, P, P, P, None, P, *dims, 0x10, None) == m["SCAN2D_E_ALIGN"]
+    assert r.scan2d_fwd(P, P, P + 2, P, P, None, P, *dims, 0x10, None) == m["SCAN2D_E_ALIGN"]
+    # bf16 buffers need 2-byte alignment only; fp32 y with OUT_F32 needs 4
+    assert r.scan2d_fwd(P, P, P, P + 1, P, None, P, *dims, 0x11, None) == m["SCAN2D_E_ALIGN"]
+    assert r.scan2d_fwd(P, P, P, P, P, None, P + 2, *dims, 0x13, None) == m["SCAN2D_E_ALIGN"]
+
+
+def test_staging_size_and_host_checks(lib):
+    m = _header_macros()
+    n = lib.scan2d_host_staging_bytes(1, 4, 8, 8, 4, 0x10)
+    # x, delta, y: 256 floats each; A 16 floats; B, C 256 floats; Dskip 4 -> rounded to 256 B
+    assert n == 256 * 4 * 3 + 256 + 256 * 4 * 2 + 256
+    assert lib.scan2d_host_staging_bytes(1, 4, 8, 8, 4, 0x1F1) == 0
+    r = lib.raw()
+    assert r.scan2d_fwd_host(P, P, P, P, P, None, P, P, n - 1, 1, 4, 8, 8, 4, 0x10, None) == m["SCAN2D_E_STAGING"]
+    assert r.scan2d_fwd_host(P, P, P, P, P, None, P, P + 16, n, 1, 4, 8, 8, 4, 0x10, None) == m["SCAN2D_E_ALIGN"]
+
+
+def test_valid_call_without_a_gpu_fails_loudly(lib):
+    """No CPU fallback: with valid arguments and no usable device the call is an error."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    m = _header_macros()
+    rc = lib.raw().scan2d_fwd(P, P, P, P, P, None, P, 1, 4, 8, 8, 4, 0x10, None)
+    assert rc == m["SCAN2D_E_DEVICE"]
+    x = torch.zeros(1, 4, 8, 8)
+    with pytest.raises(ValueError):
+        lib.scan2d_fwd(x, x, torch.zeros(4, 4), torch.zeros(1, 4, 8, 8), torch.zeros(1, 4, 8, 8))

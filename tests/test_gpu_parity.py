@@ -1,0 +1,171 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle, element by element,
+on identical seeded inputs.  Bound: |y - y_ref| <= 1e-5 (1 + |y_ref|) for fp32 inputs and
+2e-2 (1 + |y_ref|) for bf16 inputs."""
+import numpy as np
+import pytest
+
+from selective_state_space_scan2d_b200 import inputs
+from scan2d_testlib import TOL, max_violation, run_gpu, to_torch, workload, y_to_f64
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+
+def _oracle_full(oracle_mod, d, mask=None):
+    return oracle_mod.scan2d_fwd(d["x"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"],
+                                 d["orient_mask"] if mask is None else mask)
+
+
+def _check_full(oracle_mod, d, flags=None, mask=None):
+    y = y_to_f64(run_gpu(d, flags))
+    torch.cuda.synchronize()
+    ref = _oracle_full(oracle_mod, d, mask)
+    tol = TOL[d["workload"].dtype]
+    v = max_violation(y, ref, tol)
+    assert v <= 1.0, f"parity violated: worst |err| / bound = {v:.3g}"
+    from selective_state_space_scan2d_b200 import scan2d
+    assert scan2d.scan2d_get_device_error() == 0
+    return v
+
+
+# ---- small shapes covering every path (several strips, ragged tails, chains of blocks) ----
+CASES = {
+    "tiny": ("tiny", {}),
+    "f32_strips_ragged": ("tiny", dict(batch=2, channels=20, N=16, H=37, W=75)),
+    "f32_two_blocks": ("tiny", dict(batch=1, channels=9, N=16, H=21, W=200)),
+    "f32_long_chain_backpressure": ("tiny", dict(batch=1, channels=8, N=16, H=40, W=1030)),
+    "bf16_14x14": ("small", dict(batch=3, channels=19, H=14, W=14)),
+    "bf16_7x33": ("small", dict(batch=2, channels=8, H=7, W=33)),
+    "bf16_k4_in_block": ("vision", dict(batch=2, channels=12, H=24, W=40)),
+    "bf16_k4_56x56": ("vision", dict(batch=1, channels=16, H=56, W=56)),
+    "bf16_k4_across_blocks": ("vision", dict(batch=1, channels=8, H=20, W=300)),
+    "f32_k2_across_blocks": ("tiny", dict(batch=1, channels=10, N=8, H=19, W=260, orient_mask=0b1001)),
+    "f32_tr_only": ("tiny", dict(batch=1, channels=8, N=16, H=11, W=45, orient_mask=0b0010)),
+    "f32_bl_only": ("tiny", dict(batch=1, channels=8, N=16, H=11, W=45, orient_mask=0b0100)),
+    "f32_br_only_chain": ("tiny", dict(batch=1, channels=8, N=16, H=9, W=150, orient_mask=0b1000)),
+    "f32_tl_br": ("tiny", dict(batch=2, channels=5, N=4, H=13, W=29, orient_mask=0b1001)),
+    "H1": ("tiny", dict(batch=1, channels=8, N=16, H=1, W=77)),
+    "W1": ("tiny", dict(batch=1, channels=8, N=16, H=77, W=1)),
+    "H1W1": ("tiny", dict(batch=2, channels=3, N=5, H=1, W=1)),
+    "W16": ("tiny", dict(batch=1, channels=8, N=16, H=10, W=16)),
+    "W17": ("tiny", dict(batch=1, channels=8, N=16, H=10, W=17)),
+    "W128": ("tiny", dict(batch=1, channels=8, N=16, H=10, W=128)),
+    "W129": ("tiny", dict(batch=1, channels=8, N=16, H=10, W=129)),
+    "no_dskip": ("tiny", dict(batch=1, channels=8, N=16, H=12, W=40, dskip=False)),
+    "random_A": ("giga", dict(channels=8, H=48, W=100, random_A=True)),
+    "wsi_mask_recipe": ("wsi", dict(channels=16, H=40, W=56)),
+    "giga_recipe_small": ("giga", dict(channels=8, H=64, W=300)),
+}
+for n in (1, 3, 5, 8, 12, 17, 32, 33, 64):
+    CASES[f"N{n}"] = ("tiny", dict(batch=1, channels=9, N=n, H=9, W=23))
+    CASES[f"N{n}_bf16_k4"] = ("vision", dict(batch=1, channels=8, N=n, H=6, W=10))
+
+
+@pytest.mark.parametrize("case", sorted(CASES))
+def test_parity_small(oracle_mod, case):
+    name, kw = CASES[case]
+    d = inputs.make_inputs(workload(name, **kw), seed=11)
+    _check_full(oracle_mod, d)
+
+
+def test_bf16_with_fp32_output(oracle_mod):
+    from selective_state_space_scan2d_b200 import scan2d
+    d = inputs.make_inputs(workload("vision", batch=1, channels=9, H=12, W=20), seed=3)
+    y = run_gpu(d, flags=scan2d.flags_for(True, 0xF, out_f32=True))
+    assert y.dtype == torch.float32
+    ref = _oracle_full(oracle_mod, d)
+    assert max_violation(y_to_f64(y), ref, TOL["bf16"]) <= 1.0
+
+
+def test_repeat_is_bitwise_identical():
+    d = inputs.make_inputs(workload("tiny", batch=1, channels=16, N=16, H=33, W=300), seed=5)
+    a = run_gpu(d)
+    b = run_gpu(d)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_two_streams_concurrently(oracle_mod):
+    """Each stream gets its own workspace: concurrent chained launches stay correct."""
+    d1 = inputs.make_inputs(workload("tiny", batch=1, channels=8, N=16, H=30, W=400), seed=1)
+    d2 = inputs.make_inputs(workload("tiny", batch=1, channels=8, N=16, H=30, W=400), seed=2)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    with torch.cuda.stream(s1):
+        y1 = run_gpu(d1, stream=s1)
+    with torch.cuda.stream(s2):
+        y2 = run_gpu(d2, stream=s2)
+    torch.cuda.synchronize()
+    for d, y in ((d1, y1), (d2, y2)):
+        assert max_violation(y_to_f64(y), _oracle_full(oracle_mod, d), TOL["f32"]) <= 1.0
+
+
+def test_host_entry_point_matches_device():
+    from selective_state_space_scan2d_b200 import scan2d
+    d = inputs.make_inputs(workload("small", batch=4, channels=24, H=14, W=14), seed=4)
+    yd = run_gpu(d)
+    t = to_torch(d, device="cpu")
+    t = {k: (v.pin_memory() if v is not None else None) for k, v in t.items()}
+    flags = scan2d.flags_for(True, 1)
+    nbytes = scan2d.scan2d_host_staging_bytes(4, 24, 14, 14, 16, flags)
+    staging = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    yh = torch.empty(4, 24, 14, 14, dtype=torch.bfloat16).pin_memory()
+    scan2d.scan2d_fwd_host(t["x"], t["delta"], t["A"], t["B"], t["C"], t["Dskip"], yh, staging, flags)
+    torch.cuda.synchronize()
+    assert torch.equal(yh, yd.cpu())
+
+
+# ---- full-size workloads, same launch configuration as the benchmark ----------------------
+FULL = {
+    # workload: (number of whole maps checked, number of extra points)
+    "wsi": (3, 24),
+    "small": (48, 24),
+    "vision": (12, 24),
+    "giga": (2, 12),
+}
+
+
+@pytest.mark.parametrize("name", sorted(FULL))
+def test_full_size_sampled(oracle_mod, name):
+    w = inputs.WORKLOADS[name]
+    d = inputs.make_inputs(w, seed=0)
+    y = run_gpu(d)
+    torch.cuda.synchronize()
+    from selective_state_space_scan2d_b200 import scan2d
+    assert scan2d.scan2d_get_device_error() == 0
+    rng = np.random.default_rng(123)
+    nmaps, npts = FULL[name]
+    maps = {(int(rng.integers(w.batch)), int(rng.integers(w.channels))) for _ in range(nmaps)}
+    maps.add((w.batch - 1, w.channels - 1))
+    maps = sorted(maps)
+    ym = oracle_mod.scan2d_maps(d["x"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"], maps,
+                                d["orient_mask"])
+    tol = TOL[w.dtype]
+    for m, (b, ch) in enumerate(maps):
+        got = y[b, ch].to("cpu", torch.float64).numpy()
+        v = max_violation(got, ym[m], tol)
+        assert v <= 1.0, f"map {(b, ch)}: worst |err| / bound = {v:.3g}"
+    pts = [(w.batch - 1, w.channels - 1, w.H - 1, w.W - 1), (0, 0, w.H - 1, 0), (0, 0, 0, w.W - 1)]
+    for _ in range(npts):
+        pts.append((int(rng.integers(w.batch)), int(rng.integers(w.channels)),
+                    int(rng.integers(w.H)), int(rng.integers(w.W))))
+    yp = oracle_mod.scan2d_points(d["x"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"], pts,
+                                  d["orient_mask"])
+    got = np.array([float(y[p]) for p in pts])
+    v = max_violation(got, yp, tol)
+    assert v <= 1.0, f"points: worst |err| / bound = {v:.3g}"
+
+
+def test_full_size_random_A_giga_shape(oracle_mod):
+    """The kernel is not specialised to A = -(n+1): random A at the giga shape."""
+    w = inputs.WORKLOADS["giga"].scaled(random_A=True)
+    d = inputs.make_inputs(w, seed=1)
+    y = run_gpu(d)
+    torch.cuda.synchronize()
+    maps = [(0, 5), (0, 127)]
+    ym = oracle_mod.scan2d_maps(d["x"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"], maps, 1)
+    for m, (b, ch) in enumerate(maps):
+        got = y[b, ch].to("cpu", torch.float64).numpy()
+        assert max_violation(got, ym[m], TOL["f32"]) <= 1.0
