@@ -102,9 +102,11 @@ int scan2d_fwd(const void *x, const void *delta, const float *A, const void *B, 
  *   [2] threads per block               [7] 0 one orientation, 1 orientations summed in
  *   [3] dynamic shared memory bytes         shared memory, 2 one launch per orientation
  *   [4] blocks per chain (segments)     [8] states per lane   [9] workspace bytes
+ *   [10] channels per lane              [11] 1 if rows are staged by TMA (16-byte aligned
+ *                                            row stride; buffers must also be 16-byte aligned)
  * Returns 0 or the argument-check codes of scan2d_fwd.
  */
-#define SCAN2D_PLAN_FIELDS 10
+#define SCAN2D_PLAN_FIELDS 12
 int scan2d_query_plan(int batch, int channels, int H, int W, int N, unsigned flags,
                       long long *out, int n_out);
 

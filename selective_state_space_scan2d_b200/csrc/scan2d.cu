@@ -1,5 +1,7 @@
 // scan2d.cu -- C ABI of the 2D selective-scan forward: argument checks, work planning,
-// per-(device, stream) workspace, kernel dispatch.  The arithmetic is in scan2d_kernels.cuh.
+// tensor maps, per-(device, stream) workspace, kernel dispatch.  The arithmetic is in
+// scan2d_kernels.cuh.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -17,10 +19,15 @@ namespace {
 
 constexpr long long kTimeoutNs = 2000000000LL;   // bounded inter-block waits: 2 s
 constexpr size_t kAlign = 256;
+constexpr size_t kSmemBudget = 200 * 1024;       // dynamic shared memory per block we plan for
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 int popcount4(unsigned v) { return ((v >> 0) & 1) + ((v >> 1) & 1) + ((v >> 2) & 1) + ((v >> 3) & 1); }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
 
 struct Shape {
   int batch, channels, H, W, N, K;
@@ -54,64 +61,124 @@ int check_shape(int batch, int channels, int H, int W, int N, unsigned flags, Sh
   return SCAN2D_OK;
 }
 
-bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+// ---- kernel variants ------------------------------------------------------------------------
+using KernelFn = void (*)(const Params, const TmaMaps);
 
-// ---- kernel table ----------------------------------------------------------------------
-using KernelFn = void (*)(const Params);
+struct Variant {
+  int ng, g, cmax;            // states per lane, channels per lane, strip width
+  size_t tile_bytes;          // one staged strip row
+  KernelFn fn_tma, fn_plain;
+};
 
-template <typename Tin, typename Tout>
-KernelFn pick_ng(int ng) {
-  switch (ng) {
-    case 1: return scan2d_strip_kernel<Tin, Tout, 1, 16>;
-    case 2: return scan2d_strip_kernel<Tin, Tout, 2, 16>;
-    case 4: return scan2d_strip_kernel<Tin, Tout, 4, 16>;
-    case 8: return scan2d_strip_kernel<Tin, Tout, 8, 8>;
-    default: return scan2d_strip_kernel<Tin, Tout, 16, 4>;
-  }
+template <typename Tin, int NG, int G, int CMAX>
+Variant make_variant() {
+  return Variant{NG, G, CMAX, static_cast<size_t>(Layout<Tin, NG, G, CMAX>::BYTES),
+                 scan2d_kernel<Tin, NG, G, CMAX, true>, scan2d_kernel<Tin, NG, G, CMAX, false>};
 }
 
 int states_per_lane(int N) {
   int ng = 1;
-  while (ng * kStateLanes < N) ng *= 2;
+  while (ng * kQ < N) ng *= 2;
   return ng;                       // 1, 2, 4, 8 or 16 for N <= 64
 }
 
-int cmax_for(int ng) { return ng <= 4 ? 16 : (ng == 8 ? 8 : 4); }
+// G = 2 channels per lane (packed f32x2) unless the block keeps a whole-map accumulator in
+// shared memory (G = 1 halves it) or the lane already holds 16 states.
+template <typename Tin>
+Variant pick_variant_t(int ng, bool g1) {
+  constexpr bool kF32 = sizeof(Tin) == 4;
+  switch (ng) {
+    case 1: return g1 ? make_variant<Tin, 1, 1, 8>() : make_variant<Tin, 1, 2, 8>();
+    case 2: return g1 ? make_variant<Tin, 2, 1, 8>() : make_variant<Tin, 2, 2, 8>();
+    case 4: return g1 ? make_variant<Tin, 4, 1, 8>() : make_variant<Tin, 4, 2, 8>();
+    case 8:
+      if constexpr (kF32) return g1 ? make_variant<Tin, 8, 1, 4>() : make_variant<Tin, 8, 2, 4>();
+      else
+      return make_variant<Tin, 8, 1, 8>();
+    default:
+      if constexpr (kF32) return make_variant<Tin, 16, 1, 4>();
+      else
+      return make_variant<Tin, 16, 1, 8>();
+  }
+}
 
-KernelFn pick_kernel(const Shape& s, int ng) {
-  if (!s.bf16) return pick_ng<float, float>(ng);
-  if (s.out_f32) return pick_ng<uint16_t, float>(ng);
-  return pick_ng<uint16_t, uint16_t>(ng);
+Variant pick_variant(const Shape& s, int ng, bool g1) {
+  return s.bf16 ? pick_variant_t<uint16_t>(ng, g1) : pick_variant_t<float>(ng, g1);
 }
 
 // ---- work plan ---------------------------------------------------------------------------
 struct Plan {
-  int ng, cols, wpc, nseg, chains_per_block, n_cgroups, n_chains, warps;
-  size_t carry_smem;
+  Variant var;
+  int cpw, strips, wpc, nseg, chains_per_block, n_cgroups, n_chains, warps;
+  size_t carry_smem, tile_smem;
 };
 
-Plan make_plan(const Shape& s) {
+Plan make_plan(const Shape& s, int ng, bool g1, bool tma) {
   Plan pl{};
-  pl.ng = states_per_lane(s.N);
-  const int cmax = cmax_for(pl.ng);
-  pl.n_cgroups = (s.channels + kChanPerWarp - 1) / kChanPerWarp;
+  pl.var = pick_variant(s, ng, g1);
+  pl.cpw = kGroups * pl.var.g;
+  pl.n_cgroups = (s.channels + pl.cpw - 1) / pl.cpw;
   pl.n_chains = s.batch * pl.n_cgroups;
-  const int strips = (s.W + cmax - 1) / cmax;
-  if (strips == 1) {
-    pl.cols = s.W;
-    pl.wpc = 1;
+  pl.strips = (s.W + pl.var.cmax - 1) / pl.var.cmax;
+  if (pl.strips <= kMaxWarps) {
+    pl.wpc = pl.strips;
     pl.nseg = 1;
-    pl.chains_per_block = 4;
+    pl.chains_per_block = kMaxWarps / pl.wpc;
   } else {
-    pl.cols = (s.W + strips - 1) / strips;                   // balanced strips
-    const int nstrips = (s.W + pl.cols - 1) / pl.cols;
-    pl.wpc = nstrips < kMaxWarps ? nstrips : kMaxWarps;
-    pl.nseg = (nstrips + pl.wpc - 1) / pl.wpc;
+    pl.wpc = kMaxWarps;
+    pl.nseg = (pl.strips + kMaxWarps - 1) / kMaxWarps;
     pl.chains_per_block = 1;
   }
   pl.warps = pl.wpc * pl.chains_per_block;
-  pl.carry_smem = pl.wpc > 1 ? sizeof(float) * 2 * kMaxWarps * 32 * pl.ng : 0;
+  pl.carry_smem = pl.wpc > 1 ? sizeof(float) * 2 * kMaxWarps * 32 * pl.var.g * pl.var.ng : 0;
+  pl.tile_smem = static_cast<size_t>(pl.warps) * (tma ? kDepth : 1) * pl.var.tile_bytes;
   return pl;
+}
+
+// ---- tensor maps (cuTensorMapEncodeTiled through the runtime's driver entry point) -----------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// 4-D map (W, H, d2, d3) of a dense tensor with a (cmax, 1, box2, 1) box.
+bool encode_map(CUtensorMap* m, const void* base, bool bf16, int W, int H, long long d2,
+                long long d3, int cmax, int box2) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const size_t e = bf16 ? 2 : 4;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(W), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(d2), static_cast<cuuint64_t>(d3)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(W) * e,
+                                 static_cast<cuuint64_t>(W) * H * e,
+                                 static_cast<cuuint64_t>(W) * H * e * d2};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(cmax), 1u, static_cast<cuuint32_t>(box2), 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  const CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
+                        const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// TMA needs 16-byte aligned bases and row strides (W * element) that are multiples of 16 B.
+bool tma_possible(const Shape& s, const void* x, const void* delta, const void* B, const void* C) {
+  if ((static_cast<size_t>(s.W) * s.in_elem) % 16 != 0) return false;
+  return aligned(x, 16) && aligned(delta, 16) && aligned(B, 16) && aligned(C, 16);
 }
 
 // ---- per-(device, stream) workspace --------------------------------------------------------
@@ -124,7 +191,7 @@ struct Workspace {
 std::mutex g_mu;
 std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
 
-// Returns a zero-initialised (at creation) workspace of at least `bytes` bytes, or null.
+// A workspace of at least `bytes` bytes, zero-initialised when (re)created, or null.
 Workspace* get_workspace(int dev, cudaStream_t st, size_t bytes) {
   std::lock_guard<std::mutex> lk(g_mu);
   Workspace& ws = g_ws[std::make_pair(dev, st)];
@@ -135,7 +202,7 @@ Workspace* get_workspace(int dev, cudaStream_t st, size_t bytes) {
       ws.ptr = nullptr;
       ws.bytes = 0;
     }
-    size_t want = round_up(bytes, 1 << 20);
+    const size_t want = round_up(bytes, 1 << 20);
     if (cudaMalloc(&ws.ptr, want) != cudaSuccess) {
       cudaGetLastError();
       ws.ptr = nullptr;
@@ -152,18 +219,6 @@ Workspace* get_workspace(int dev, cudaStream_t st, size_t bytes) {
   return &ws;
 }
 
-int launch(KernelFn fn, const Plan& pl, Params prm, size_t smem, int grid, cudaStream_t st) {
-  if (smem > 48 * 1024) {
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess) {
-      cudaGetLastError();
-      return SCAN2D_E_LAUNCH;
-    }
-  }
-  fn<<<grid, pl.warps * 32, smem, st>>>(prm);
-  if (cudaGetLastError() != cudaSuccess) return SCAN2D_E_LAUNCH;
-  return SCAN2D_OK;
-}
-
 int device_ok(int* dev, int* nsm) {
   if (cudaGetDevice(dev) != cudaSuccess) { cudaGetLastError(); return SCAN2D_E_DEVICE; }
   int major = 0;
@@ -176,34 +231,54 @@ int device_ok(int* dev, int* nsm) {
   return SCAN2D_OK;
 }
 
-}  // namespace
-
 // Everything a call of this shape launches, without touching memory.
 struct CallPlan {
   Plan pl;
-  KernelFn fn;
+  bool tma;
   int codes[4], nk;
   bool smem_multi, global_multi, need_yacc_ws, need_ws;
   int yacc_stride, grid, launches;
   size_t smem, off_ctrl, off_flags, off_acks, off_carry, off_yacc, ws_bytes;
 };
 
-CallPlan plan_call(const Shape& s) {
+CallPlan plan_call(const Shape& s, bool tma) {
   CallPlan cp{};
-  cp.pl = make_plan(s);
-  const Plan& pl = cp.pl;
-  cp.fn = pick_kernel(s, pl.ng);
+  cp.tma = tma;
+  const int ng = states_per_lane(s.N);
   cp.nk = 0;
   for (int o = 0; o < 4; ++o)
     if (s.orient & (1u << o)) cp.codes[cp.nk++] = o;
+
+  // several orientations: sum them in a shared-memory accumulator when a block can hold
+  // whole maps of its channels (G = 1 channel per lane keeps it small); otherwise one
+  // launch per orientation with an fp32 accumulator in global memory.
   const size_t HW = static_cast<size_t>(s.H) * s.W;
-  size_t yacc_smem = ~size_t(0);
-  cp.yacc_stride = 0;
-  if (HW <= (1u << 20)) {
-    cp.yacc_stride = static_cast<int>(round_up(HW, 32) + 4);          // +4: spread the banks
-    yacc_smem = sizeof(float) * static_cast<size_t>(pl.chains_per_block) * kChanPerWarp * cp.yacc_stride;
+  cp.smem_multi = false;
+  if (s.K > 1 && HW <= (1u << 20)) {
+    Plan p1 = make_plan(s, ng, true, tma);
+    const int stride = static_cast<int>(round_up(HW, 32) + 4);        // +4: spread the banks
+    if (p1.nseg == 1) {
+      const size_t per_chain = sizeof(float) * p1.cpw * stride;
+      const size_t tile_per_chain = p1.tile_smem / p1.chains_per_block;
+      int cpb = p1.chains_per_block;
+      while (cpb > 1 && p1.carry_smem + (tile_per_chain + per_chain) * cpb > kSmemBudget) --cpb;
+      if (p1.carry_smem + (tile_per_chain + per_chain) * cpb <= kSmemBudget) {
+        p1.chains_per_block = cpb;
+        p1.warps = p1.wpc * cpb;
+        p1.tile_smem = tile_per_chain * cpb;
+        cp.pl = p1;
+        cp.smem_multi = true;
+        cp.yacc_stride = stride;
+        cp.smem = p1.carry_smem + p1.tile_smem + per_chain * cpb;
+      }
+    }
   }
-  cp.smem_multi = s.K > 1 && pl.nseg == 1 && yacc_smem != ~size_t(0) && pl.carry_smem + yacc_smem <= 200 * 1024;
+  if (!cp.smem_multi) {
+    cp.pl = make_plan(s, ng, ng >= 16, tma);
+    cp.yacc_stride = 0;
+    cp.smem = cp.pl.carry_smem + cp.pl.tile_smem;
+  }
+  const Plan& pl = cp.pl;
   cp.global_multi = s.K > 1 && !cp.smem_multi;
   cp.need_yacc_ws = cp.global_multi && !s.out_f32;
   const size_t items = static_cast<size_t>(pl.n_chains) * pl.nseg;
@@ -211,15 +286,27 @@ CallPlan plan_call(const Shape& s) {
   cp.off_flags = kAlign;
   cp.off_acks = cp.off_flags + round_up(items * 8, kAlign);
   cp.off_carry = cp.off_acks + round_up(items * 8, kAlign);
-  cp.off_yacc = cp.off_carry + round_up(items * kRing * 32 * pl.ng * sizeof(float), kAlign);
+  cp.off_yacc = cp.off_carry + round_up(items * kRing * 32 * pl.var.g * pl.var.ng * sizeof(float), kAlign);
   cp.ws_bytes = cp.off_yacc + (cp.need_yacc_ws ? s.xy_count * sizeof(float) : 0);
   cp.need_ws = pl.nseg > 1 || cp.need_yacc_ws;
   if (!cp.need_ws) cp.ws_bytes = 0;
   cp.grid = pl.nseg > 1 ? pl.n_chains * pl.nseg
                         : (pl.n_chains + pl.chains_per_block - 1) / pl.chains_per_block;
-  cp.smem = pl.carry_smem + (cp.smem_multi ? yacc_smem : 0);
   cp.launches = cp.global_multi ? cp.nk : 1;
   return cp;
+}
+
+int launch(KernelFn fn, int threads, const Params& prm, const TmaMaps& tm, size_t smem, int grid,
+           cudaStream_t st) {
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess) {
+      cudaGetLastError();
+      return SCAN2D_E_LAUNCH;
+    }
+  }
+  fn<<<grid, threads, smem, st>>>(prm, tm);
+  if (cudaGetLastError() != cudaSuccess) return SCAN2D_E_LAUNCH;
+  return SCAN2D_OK;
 }
 
 int forward(const void* x, const void* delta, const float* A, const void* B, const void* C,
@@ -236,25 +323,41 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
   rc = device_ok(&dev, &nsm);
   if (rc) return rc;
 
-  const CallPlan cp = plan_call(s);
+  // tensor maps when the layout allows TMA, else the plain-load variant
+  TmaMaps tm;
+  std::memset(&tm, 0, sizeof tm);
+  bool tma = tma_possible(s, x, delta, B, C);
+  CallPlan cp = plan_call(s, tma);
+  if (tma) {
+    const Plan& p0 = cp.pl;
+    const int nb = kQ * p0.var.ng;
+    tma = encode_map(&tm.x, x, s.bf16, W, H, channels, batch, p0.var.cmax, p0.cpw) &&
+          encode_map(&tm.d, delta, s.bf16, W, H, channels, batch, p0.var.cmax, p0.cpw) &&
+          encode_map(&tm.b, B, s.bf16, W, H, N, static_cast<long long>(batch) * s.K, p0.var.cmax, nb) &&
+          encode_map(&tm.c, C, s.bf16, W, H, N, static_cast<long long>(batch) * s.K, p0.var.cmax, nb);
+    if (!tma) cp = plan_call(s, false);
+  }
   const Plan& pl = cp.pl;
+  const KernelFn fn = tma ? pl.var.fn_tma : pl.var.fn_plain;
 
   Params prm;
   std::memset(&prm, 0, sizeof prm);
   prm.x = x; prm.delta = delta; prm.A = A; prm.B = B; prm.C = C; prm.Dskip = Dskip; prm.y = y;
   prm.batch = batch; prm.channels = channels; prm.H = H; prm.W = W; prm.N = N; prm.K = s.K;
   prm.n_cgroups = pl.n_cgroups; prm.n_chains = pl.n_chains;
-  prm.cols_per_warp = pl.cols; prm.wpc = pl.wpc; prm.chains_per_block = pl.chains_per_block;
+  prm.strips = pl.strips; prm.wpc = pl.wpc; prm.chains_per_block = pl.chains_per_block;
   prm.nseg = pl.nseg;
   prm.timeout_ns = kTimeoutNs;
   prm.yacc_stride = cp.yacc_stride;
+  prm.out_f32 = s.out_f32 ? 1 : 0;
+  prm.vec_store = (W % 4 == 0) && aligned(y, s.out_f32 ? 16 : 8);
 
   Workspace* ws = nullptr;
   if (cp.need_ws) {
     if (pl.nseg > 1) {
       // a chain's blocks must be able to be resident together (producer back-pressure)
       int per_sm = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, cp.fn, pl.warps * 32, pl.carry_smem) != cudaSuccess) {
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, pl.warps * 32, cp.smem) != cudaSuccess) {
         cudaGetLastError();
         return SCAN2D_E_LAUNCH;
       }
@@ -277,12 +380,13 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
     return ++ws->gen;
   };
 
+  const int threads = pl.warps * 32;
   if (!cp.global_multi) {
     prm.mode = cp.smem_multi ? kSmemMulti : kSingle;
     prm.orient_count = cp.smem_multi ? cp.nk : 1;
     for (int k = 0; k < prm.orient_count; ++k) { prm.orient_code[k] = cp.codes[k]; prm.orient_k[k] = k; }
     prm.gen = next_gen();
-    return launch(cp.fn, pl, prm, cp.smem, cp.grid, st);
+    return launch(fn, threads, prm, tm, cp.smem, cp.grid, st);
   }
   for (int k = 0; k < cp.nk; ++k) {
     prm.mode = k == 0 ? kGlobalFirst : (k == cp.nk - 1 ? kGlobalLast : kGlobalMid);
@@ -290,7 +394,7 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
     prm.orient_code[0] = cp.codes[k];
     prm.orient_k[0] = k;
     prm.gen = next_gen();
-    rc = launch(cp.fn, pl, prm, cp.smem, cp.grid, st);
+    rc = launch(fn, threads, prm, tm, cp.smem, cp.grid, st);
     if (rc) return rc;
   }
   return SCAN2D_OK;
@@ -314,11 +418,13 @@ int scan2d_query_plan(int batch, int channels, int H, int W, int N, unsigned fla
   const int rc = scan2d::check_shape(batch, channels, H, W, N, flags, &s);
   if (rc) return rc;
   if (!out) return SCAN2D_E_NULL;
-  const scan2d::CallPlan cp = scan2d::plan_call(s);
+  // the layout decides TMA; with 16-byte aligned buffers only the row stride matters
+  const bool tma = (static_cast<size_t>(W) * s.in_elem) % 16 == 0;
+  const scan2d::CallPlan cp = scan2d::plan_call(s, tma);
   const long long v[SCAN2D_PLAN_FIELDS] = {
       cp.launches, cp.grid, cp.pl.warps * 32, static_cast<long long>(cp.smem), cp.pl.nseg,
-      cp.pl.cols, cp.pl.wpc, cp.smem_multi ? 1 : (cp.global_multi ? 2 : 0), cp.pl.ng,
-      static_cast<long long>(cp.ws_bytes)};
+      cp.pl.var.cmax, cp.pl.wpc, cp.smem_multi ? 1 : (cp.global_multi ? 2 : 0), cp.pl.var.ng,
+      static_cast<long long>(cp.ws_bytes), cp.pl.var.g, tma ? 1 : 0};
   for (int k = 0; k < n_out && k < SCAN2D_PLAN_FIELDS; ++k) out[k] = v[k];
   return SCAN2D_OK;
 }
@@ -413,6 +519,6 @@ const char* scan2d_strerror(int code) {
   }
 }
 
-int scan2d_version(void) { return 100; }
+int scan2d_version(void) { return 200; }
 
 }  // extern "C"

@@ -39,6 +39,22 @@ def max_violation(y, ref, tol):
     return float(np.max(np.abs(y - ref) / (tol * (1.0 + np.abs(ref)))))
 
 
+def assert_parity(y, ref, tol, label=""):
+    """Element-wise bound |y - ref| <= tol (1 + |ref|), with a diagnosis on failure."""
+    y = np.asarray(y, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    ratio = np.abs(y - ref) / (tol * (1.0 + np.abs(ref)))
+    worst = float(np.nanmax(ratio)) if ratio.size else 0.0
+    if not (worst <= 1.0) or not np.all(np.isfinite(y)):
+        bad = ratio > 1.0
+        idx = np.unravel_index(int(np.nanargmax(ratio)), ratio.shape)
+        raise AssertionError(
+            f"{label}: parity violated at {int(bad.sum())} of {ratio.size} elements; worst "
+            f"{worst:.3g}x the bound at {tuple(int(v) for v in idx)}: got {y[idx]!r}, "
+            f"want {ref[idx]!r}; non-finite outputs: {int((~np.isfinite(y)).sum())}")
+    return worst
+
+
 def workload(name, **kw):
     w = inputs.WORKLOADS[name]
     return w.scaled(**kw) if kw else w

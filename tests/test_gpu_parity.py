@@ -5,7 +5,8 @@ import numpy as np
 import pytest
 
 from selective_state_space_scan2d_b200 import inputs
-from scan2d_testlib import TOL, max_violation, run_gpu, to_torch, workload, y_to_f64
+from scan2d_cases import CASES
+from scan2d_testlib import TOL, assert_parity, max_violation, run_gpu, to_torch, workload, y_to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -23,45 +24,10 @@ def _check_full(oracle_mod, d, flags=None, mask=None):
     y = y_to_f64(run_gpu(d, flags))
     torch.cuda.synchronize()
     ref = _oracle_full(oracle_mod, d, mask)
-    tol = TOL[d["workload"].dtype]
-    v = max_violation(y, ref, tol)
-    assert v <= 1.0, f"parity violated: worst |err| / bound = {v:.3g}"
+    v = assert_parity(y, ref, TOL[d["workload"].dtype], d["workload"].name)
     from selective_state_space_scan2d_b200 import scan2d
     assert scan2d.scan2d_get_device_error() == 0
     return v
-
-
-# ---- small shapes covering every path (several strips, ragged tails, chains of blocks) ----
-CASES = {
-    "tiny": ("tiny", {}),
-    "f32_strips_ragged": ("tiny", dict(batch=2, channels=20, N=16, H=37, W=75)),
-    "f32_two_blocks": ("tiny", dict(batch=1, channels=9, N=16, H=21, W=200)),
-    "f32_long_chain_backpressure": ("tiny", dict(batch=1, channels=8, N=16, H=40, W=1030)),
-    "bf16_14x14": ("small", dict(batch=3, channels=19, H=14, W=14)),
-    "bf16_7x33": ("small", dict(batch=2, channels=8, H=7, W=33)),
-    "bf16_k4_in_block": ("vision", dict(batch=2, channels=12, H=24, W=40)),
-    "bf16_k4_56x56": ("vision", dict(batch=1, channels=16, H=56, W=56)),
-    "bf16_k4_across_blocks": ("vision", dict(batch=1, channels=8, H=20, W=300)),
-    "f32_k2_across_blocks": ("tiny", dict(batch=1, channels=10, N=8, H=19, W=260, orient_mask=0b1001)),
-    "f32_tr_only": ("tiny", dict(batch=1, channels=8, N=16, H=11, W=45, orient_mask=0b0010)),
-    "f32_bl_only": ("tiny", dict(batch=1, channels=8, N=16, H=11, W=45, orient_mask=0b0100)),
-    "f32_br_only_chain": ("tiny", dict(batch=1, channels=8, N=16, H=9, W=150, orient_mask=0b1000)),
-    "f32_tl_br": ("tiny", dict(batch=2, channels=5, N=4, H=13, W=29, orient_mask=0b1001)),
-    "H1": ("tiny", dict(batch=1, channels=8, N=16, H=1, W=77)),
-    "W1": ("tiny", dict(batch=1, channels=8, N=16, H=77, W=1)),
-    "H1W1": ("tiny", dict(batch=2, channels=3, N=5, H=1, W=1)),
-    "W16": ("tiny", dict(batch=1, channels=8, N=16, H=10, W=16)),
-    "W17": ("tiny", dict(batch=1, channels=8, N=16, H=10, W=17)),
-    "W128": ("tiny", dict(batch=1, channels=8, N=16, H=10, W=128)),
-    "W129": ("tiny", dict(batch=1, channels=8, N=16, H=10, W=129)),
-    "no_dskip": ("tiny", dict(batch=1, channels=8, N=16, H=12, W=40, dskip=False)),
-    "random_A": ("giga", dict(channels=8, H=48, W=100, random_A=True)),
-    "wsi_mask_recipe": ("wsi", dict(channels=16, H=40, W=56)),
-    "giga_recipe_small": ("giga", dict(channels=8, H=64, W=300)),
-}
-for n in (1, 3, 5, 8, 12, 17, 32, 33, 64):
-    CASES[f"N{n}"] = ("tiny", dict(batch=1, channels=9, N=n, H=9, W=23))
-    CASES[f"N{n}_bf16_k4"] = ("vision", dict(batch=1, channels=8, N=n, H=6, W=10))
 
 
 @pytest.mark.parametrize("case", sorted(CASES))
@@ -145,8 +111,7 @@ def test_full_size_sampled(oracle_mod, name):
     tol = TOL[w.dtype]
     for m, (b, ch) in enumerate(maps):
         got = y[b, ch].to("cpu", torch.float64).numpy()
-        v = max_violation(got, ym[m], tol)
-        assert v <= 1.0, f"map {(b, ch)}: worst |err| / bound = {v:.3g}"
+        assert_parity(got, ym[m], tol, f"{name} map {(b, ch)}")
     pts = [(w.batch - 1, w.channels - 1, w.H - 1, w.W - 1), (0, 0, w.H - 1, 0), (0, 0, 0, w.W - 1)]
     for _ in range(npts):
         pts.append((int(rng.integers(w.batch)), int(rng.integers(w.channels)),
@@ -154,8 +119,7 @@ def test_full_size_sampled(oracle_mod, name):
     yp = oracle_mod.scan2d_points(d["x"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"], pts,
                                   d["orient_mask"])
     got = np.array([float(y[p]) for p in pts])
-    v = max_violation(got, yp, tol)
-    assert v <= 1.0, f"points: worst |err| / bound = {v:.3g}"
+    assert_parity(got, yp, tol, f"{name} points")
 
 
 def test_full_size_random_A_giga_shape(oracle_mod):
@@ -168,4 +132,4 @@ def test_full_size_random_A_giga_shape(oracle_mod):
     ym = oracle_mod.scan2d_maps(d["x"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"], maps, 1)
     for m, (b, ch) in enumerate(maps):
         got = y[b, ch].to("cpu", torch.float64).numpy()
-        assert max_violation(got, ym[m], TOL["f32"]) <= 1.0
+        assert_parity(got, ym[m], TOL["f32"], f"random-A map {(b, ch)}")
