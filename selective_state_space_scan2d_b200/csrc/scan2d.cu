@@ -182,38 +182,49 @@ bool tma_possible(const Shape& s, const void* x, const void* delta, const void* 
 }
 
 // ---- per-(device, stream) workspace --------------------------------------------------------
+// Layout: [control words: 256 B][flags: cap_items u64][acks: cap_items u64][carry ring ...]
+// [fp32 accumulator ...].  The flag and ack words keep their place for the life of the
+// allocation (only generation-tagged values are ever written there), so a later call of
+// another shape can never read an earlier call's carry values as flags.  The region is
+// reallocated, zeroed, when a call needs more items than it holds.
 struct Workspace {
   void* ptr = nullptr;
   size_t bytes = 0;
+  size_t cap_items = 0;
   unsigned long long gen = 0;
 };
 
 std::mutex g_mu;
 std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
 
-// A workspace of at least `bytes` bytes, zero-initialised when (re)created, or null.
-Workspace* get_workspace(int dev, cudaStream_t st, size_t bytes) {
+size_t sync_bytes(size_t items) { return kAlign + round_up(items * 8, kAlign) * 2; }
+
+// A workspace whose flag region holds `items` items and whose tail after it holds `tail`
+// bytes, zero-initialised when (re)created, or null.
+Workspace* get_workspace(int dev, cudaStream_t st, size_t items, size_t tail) {
   std::lock_guard<std::mutex> lk(g_mu);
   Workspace& ws = g_ws[std::make_pair(dev, st)];
-  if (ws.bytes < bytes) {
+  if (ws.cap_items < items || ws.bytes < sync_bytes(ws.cap_items) + tail) {
+    size_t cap = ws.cap_items;
+    if (cap < items) cap = items > 2 * cap ? items : 2 * cap;
     if (ws.ptr != nullptr) {
       if (cudaStreamSynchronize(st) != cudaSuccess) return nullptr;
       cudaFree(ws.ptr);
-      ws.ptr = nullptr;
-      ws.bytes = 0;
+      ws = Workspace{};
     }
-    const size_t want = round_up(bytes, 1 << 20);
+    const size_t want = round_up(sync_bytes(cap) + tail, 1 << 20);
     if (cudaMalloc(&ws.ptr, want) != cudaSuccess) {
       cudaGetLastError();
-      ws.ptr = nullptr;
+      ws = Workspace{};
       return nullptr;
     }
     if (cudaMemsetAsync(ws.ptr, 0, want, st) != cudaSuccess) {
       cudaFree(ws.ptr);
-      ws.ptr = nullptr;
+      ws = Workspace{};
       return nullptr;
     }
     ws.bytes = want;
+    ws.cap_items = cap;
     ws.gen = 0;
   }
   return &ws;
@@ -238,7 +249,7 @@ struct CallPlan {
   int codes[4], nk;
   bool smem_multi, global_multi, need_yacc_ws, need_ws;
   int yacc_stride, grid, launches;
-  size_t smem, off_ctrl, off_flags, off_acks, off_carry, off_yacc, ws_bytes;
+  size_t smem, items, carry_bytes, yacc_bytes, ws_bytes;
 };
 
 CallPlan plan_call(const Shape& s, bool tma) {
@@ -281,29 +292,31 @@ CallPlan plan_call(const Shape& s, bool tma) {
   const Plan& pl = cp.pl;
   cp.global_multi = s.K > 1 && !cp.smem_multi;
   cp.need_yacc_ws = cp.global_multi && !s.out_f32;
-  const size_t items = static_cast<size_t>(pl.n_chains) * pl.nseg;
-  cp.off_ctrl = 0;
-  cp.off_flags = kAlign;
-  cp.off_acks = cp.off_flags + round_up(items * 8, kAlign);
-  cp.off_carry = cp.off_acks + round_up(items * 8, kAlign);
-  cp.off_yacc = cp.off_carry + round_up(items * kRing * 32 * pl.var.g * pl.var.ng * sizeof(float), kAlign);
-  cp.ws_bytes = cp.off_yacc + (cp.need_yacc_ws ? s.xy_count * sizeof(float) : 0);
+  cp.items = static_cast<size_t>(pl.n_chains) * pl.nseg;
+  cp.carry_bytes = pl.nseg > 1 ? round_up(cp.items * kRing * 32 * pl.var.g * pl.var.ng * sizeof(float), kAlign) : 0;
+  cp.yacc_bytes = cp.need_yacc_ws ? s.xy_count * sizeof(float) : 0;
   cp.need_ws = pl.nseg > 1 || cp.need_yacc_ws;
-  if (!cp.need_ws) cp.ws_bytes = 0;
+  cp.ws_bytes = cp.need_ws ? sync_bytes(cp.items) + cp.carry_bytes + cp.yacc_bytes : 0;
   cp.grid = pl.nseg > 1 ? pl.n_chains * pl.nseg
                         : (pl.n_chains + pl.chains_per_block - 1) / pl.chains_per_block;
   cp.launches = cp.global_multi ? cp.nk : 1;
   return cp;
 }
 
+// Raises the kernel's dynamic shared-memory limit when it needs more than the default 48 KB
+// (before occupancy queries and launches).
+bool allow_smem(KernelFn fn, size_t smem) {
+  if (smem <= 48 * 1024) return true;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return true;
+}
+
 int launch(KernelFn fn, int threads, const Params& prm, const TmaMaps& tm, size_t smem, int grid,
            cudaStream_t st) {
-  if (smem > 48 * 1024) {
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess) {
-      cudaGetLastError();
-      return SCAN2D_E_LAUNCH;
-    }
-  }
+  if (!allow_smem(fn, smem)) return SCAN2D_E_LAUNCH;
   fn<<<grid, threads, smem, st>>>(prm, tm);
   if (cudaGetLastError() != cudaSuccess) return SCAN2D_E_LAUNCH;
   return SCAN2D_OK;
@@ -357,20 +370,22 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
     if (pl.nseg > 1) {
       // a chain's blocks must be able to be resident together (producer back-pressure)
       int per_sm = 0;
+      if (!allow_smem(fn, cp.smem)) return SCAN2D_E_LAUNCH;
       if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, pl.warps * 32, cp.smem) != cudaSuccess) {
         cudaGetLastError();
         return SCAN2D_E_LAUNCH;
       }
       if (static_cast<long long>(per_sm) * nsm < pl.nseg) return SCAN2D_E_DIMS;
     }
-    ws = get_workspace(dev, st, cp.ws_bytes);
+    ws = get_workspace(dev, st, cp.items, cp.carry_bytes + cp.yacc_bytes);
     if (!ws) return SCAN2D_E_NOMEM;
     char* base = static_cast<char*>(ws->ptr);
-    prm.ctrl = reinterpret_cast<unsigned long long*>(base + cp.off_ctrl);
-    prm.flags = reinterpret_cast<unsigned long long*>(base + cp.off_flags);
-    prm.acks = reinterpret_cast<unsigned long long*>(base + cp.off_acks);
-    prm.carry = reinterpret_cast<float*>(base + cp.off_carry);
-    if (cp.need_yacc_ws) prm.yacc = reinterpret_cast<float*>(base + cp.off_yacc);
+    const size_t cap = ws->cap_items;
+    prm.ctrl = reinterpret_cast<unsigned long long*>(base);
+    prm.flags = reinterpret_cast<unsigned long long*>(base + kAlign);
+    prm.acks = reinterpret_cast<unsigned long long*>(base + kAlign + round_up(cap * 8, kAlign));
+    prm.carry = reinterpret_cast<float*>(base + sync_bytes(cap));
+    if (cp.need_yacc_ws) prm.yacc = reinterpret_cast<float*>(base + sync_bytes(cap) + cp.carry_bytes);
   }
   if (cp.global_multi && s.out_f32) prm.yacc = static_cast<float*>(y);
 

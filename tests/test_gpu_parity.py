@@ -133,3 +133,19 @@ def test_full_size_random_A_giga_shape(oracle_mod):
     for m, (b, ch) in enumerate(maps):
         got = y[b, ch].to("cpu", torch.float64).numpy()
         assert_parity(got, ym[m], TOL["f32"], f"random-A map {(b, ch)}")
+
+
+def test_workspace_reuse_across_shapes(oracle_mod):
+    """A chained call after calls of other shapes on the same stream: the earlier calls'
+    carry values must never be read as the later call's flags."""
+    s = torch.cuda.Stream()
+    big = inputs.make_inputs(workload("tiny", batch=1, channels=16, N=16, H=24, W=1024), seed=21)
+    small = inputs.make_inputs(workload("tiny", batch=1, channels=32, N=16, H=24, W=200), seed=22)
+    with torch.cuda.stream(s):
+        run_gpu(big, stream=s)
+        run_gpu(small, stream=s)
+        y = run_gpu(big, stream=s)
+    s.synchronize()
+    from selective_state_space_scan2d_b200 import scan2d
+    assert scan2d.scan2d_get_device_error(s) == 0
+    assert_parity(y_to_f64(y), _oracle_full(oracle_mod, big), TOL["f32"], "reuse")
