@@ -104,9 +104,11 @@ int scan2d_fwd(const void *x, const void *delta, const float *A, const void *B, 
  *   [4] blocks per chain (segments)     [8] states per lane   [9] workspace bytes
  *   [10] channels per lane              [11] 1 if rows are staged by TMA (16-byte aligned
  *                                            row stride; buffers must also be 16-byte aligned)
+ *   [12] how the blocks of a chain hand carries over: 0 one block per chain, 1 thread-block
+ *        cluster (distributed shared memory), 2 ring in the internal global workspace
  * Returns 0 or the argument-check codes of scan2d_fwd.
  */
-#define SCAN2D_PLAN_FIELDS 12
+#define SCAN2D_PLAN_FIELDS 13
 int scan2d_query_plan(int batch, int channels, int H, int W, int N, unsigned flags,
                       long long *out, int n_out);
 

@@ -67,12 +67,14 @@ using KernelFn = void (*)(const Params, const TmaMaps);
 struct Variant {
   int ng, g, cmax;            // states per lane, channels per lane, strip width
   size_t tile_bytes;          // one staged strip row
+  size_t carry_slot_bytes;    // one carry row of a warp
   KernelFn fn_tma, fn_plain;
 };
 
 template <typename Tin, int NG, int G, int CMAX>
 Variant make_variant() {
-  return Variant{NG, G, CMAX, static_cast<size_t>(Layout<Tin, NG, G, CMAX>::BYTES),
+  using L = Layout<Tin, NG, G, CMAX>;
+  return Variant{NG, G, CMAX, static_cast<size_t>(L::TILE_BYTES), static_cast<size_t>(L::CARRY_SLOT_BYTES),
                  scan2d_kernel<Tin, NG, G, CMAX, true>, scan2d_kernel<Tin, NG, G, CMAX, false>};
 }
 
@@ -110,8 +112,10 @@ Variant pick_variant(const Shape& s, int ng, bool g1) {
 struct Plan {
   Variant var;
   int cpw, strips, wpc, nseg, chains_per_block, n_cgroups, n_chains, warps;
-  size_t carry_smem, tile_smem;
+  size_t carry_smem, tile_smem;   // carry rings and tile rings of all warps of a block
 };
+
+constexpr int kMaxCluster = 16;   // blocks of a chain that can share distributed shared memory
 
 Plan make_plan(const Shape& s, int ng, bool g1, bool tma) {
   Plan pl{};
@@ -130,7 +134,7 @@ Plan make_plan(const Shape& s, int ng, bool g1, bool tma) {
     pl.chains_per_block = 1;
   }
   pl.warps = pl.wpc * pl.chains_per_block;
-  pl.carry_smem = pl.wpc > 1 ? sizeof(float) * 2 * kMaxWarps * 32 * pl.var.g * pl.var.ng : 0;
+  pl.carry_smem = static_cast<size_t>(pl.warps) * kCarryRing * pl.var.carry_slot_bytes;
   pl.tile_smem = static_cast<size_t>(pl.warps) * (tma ? kDepth : 1) * pl.var.tile_bytes;
   return pl;
 }
@@ -248,11 +252,11 @@ struct CallPlan {
   bool tma;
   int codes[4], nk;
   bool smem_multi, global_multi, need_yacc_ws, need_ws;
-  int yacc_stride, grid, launches;
+  int link, yacc_stride, grid, launches;
   size_t smem, items, carry_bytes, yacc_bytes, ws_bytes;
 };
 
-CallPlan plan_call(const Shape& s, bool tma) {
+CallPlan plan_call(const Shape& s, bool tma, bool cluster_ok) {
   CallPlan cp{};
   cp.tma = tma;
   const int ng = states_per_lane(s.N);
@@ -269,18 +273,19 @@ CallPlan plan_call(const Shape& s, bool tma) {
     Plan p1 = make_plan(s, ng, true, tma);
     const int stride = static_cast<int>(round_up(HW, 32) + 4);        // +4: spread the banks
     if (p1.nseg == 1) {
-      const size_t per_chain = sizeof(float) * p1.cpw * stride;
-      const size_t tile_per_chain = p1.tile_smem / p1.chains_per_block;
+      const size_t per_chain = sizeof(float) * p1.cpw * stride +
+                               (p1.tile_smem + p1.carry_smem) / p1.chains_per_block;
       int cpb = p1.chains_per_block;
-      while (cpb > 1 && p1.carry_smem + (tile_per_chain + per_chain) * cpb > kSmemBudget) --cpb;
-      if (p1.carry_smem + (tile_per_chain + per_chain) * cpb <= kSmemBudget) {
+      while (cpb > 1 && per_chain * cpb > kSmemBudget) --cpb;
+      if (per_chain * cpb <= kSmemBudget) {
+        p1.tile_smem = p1.tile_smem / p1.chains_per_block * cpb;
+        p1.carry_smem = p1.carry_smem / p1.chains_per_block * cpb;
         p1.chains_per_block = cpb;
         p1.warps = p1.wpc * cpb;
-        p1.tile_smem = tile_per_chain * cpb;
         cp.pl = p1;
         cp.smem_multi = true;
         cp.yacc_stride = stride;
-        cp.smem = p1.carry_smem + p1.tile_smem + per_chain * cpb;
+        cp.smem = per_chain * cpb;
       }
     }
   }
@@ -290,13 +295,15 @@ CallPlan plan_call(const Shape& s, bool tma) {
     cp.smem = cp.pl.carry_smem + cp.pl.tile_smem;
   }
   const Plan& pl = cp.pl;
+  cp.link = pl.nseg == 1 ? kLinkNone : (cluster_ok && pl.nseg <= kMaxCluster ? kLinkCluster : kLinkGlobal);
   cp.global_multi = s.K > 1 && !cp.smem_multi;
   cp.need_yacc_ws = cp.global_multi && !s.out_f32;
   cp.items = static_cast<size_t>(pl.n_chains) * pl.nseg;
-  cp.carry_bytes = pl.nseg > 1 ? round_up(cp.items * kRing * 32 * pl.var.g * pl.var.ng * sizeof(float), kAlign) : 0;
+  cp.carry_bytes = cp.link == kLinkGlobal
+                       ? round_up(cp.items * kRing * 32 * pl.var.g * pl.var.ng * sizeof(float), kAlign) : 0;
   cp.yacc_bytes = cp.need_yacc_ws ? s.xy_count * sizeof(float) : 0;
-  cp.need_ws = pl.nseg > 1 || cp.need_yacc_ws;
-  cp.ws_bytes = cp.need_ws ? sync_bytes(cp.items) + cp.carry_bytes + cp.yacc_bytes : 0;
+  cp.need_ws = cp.link == kLinkGlobal || cp.need_yacc_ws;
+  cp.ws_bytes = cp.need_ws ? sync_bytes(cp.link == kLinkGlobal ? cp.items : 0) + cp.carry_bytes + cp.yacc_bytes : 0;
   cp.grid = pl.nseg > 1 ? pl.n_chains * pl.nseg
                         : (pl.n_chains + pl.chains_per_block - 1) / pl.chains_per_block;
   cp.launches = cp.global_multi ? cp.nk : 1;
@@ -306,7 +313,8 @@ CallPlan plan_call(const Shape& s, bool tma) {
 // Raises the kernel's dynamic shared-memory limit when it needs more than the default 48 KB
 // (before occupancy queries and launches).
 bool allow_smem(KernelFn fn, size_t smem) {
-  if (smem <= 48 * 1024) return true;
+  // static shared memory (barriers) counts against the same 48 KB default
+  if (smem + 4096 <= 48 * 1024) return true;
   if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess) {
     cudaGetLastError();
     return false;
@@ -315,11 +323,57 @@ bool allow_smem(KernelFn fn, size_t smem) {
 }
 
 int launch(KernelFn fn, int threads, const Params& prm, const TmaMaps& tm, size_t smem, int grid,
-           cudaStream_t st) {
+           int cluster, cudaStream_t st) {
   if (!allow_smem(fn, smem)) return SCAN2D_E_LAUNCH;
-  fn<<<grid, threads, smem, st>>>(prm, tm);
+  if (cluster <= 1) {
+    fn<<<grid, threads, smem, st>>>(prm, tm);
+  } else {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(threads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, fn, prm, tm) != cudaSuccess) {
+      cudaGetLastError();
+      return SCAN2D_E_LAUNCH;
+    }
+  }
   if (cudaGetLastError() != cudaSuccess) return SCAN2D_E_LAUNCH;
   return SCAN2D_OK;
+}
+
+// Can clusters of `nseg` blocks of this kernel be resident at all on this device?
+bool cluster_fits(KernelFn fn, int threads, size_t smem, int nseg) {
+  if (nseg > kMaxCluster) return false;
+  if (!allow_smem(fn, smem)) return false;
+  if (nseg > 8 && cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nseg, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = nseg;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return n > 0;
 }
 
 int forward(const void* x, const void* delta, const float* A, const void* B, const void* C,
@@ -340,7 +394,7 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
   TmaMaps tm;
   std::memset(&tm, 0, sizeof tm);
   bool tma = tma_possible(s, x, delta, B, C);
-  CallPlan cp = plan_call(s, tma);
+  CallPlan cp = plan_call(s, tma, true);
   if (tma) {
     const Plan& p0 = cp.pl;
     const int nb = kQ * p0.var.ng;
@@ -348,8 +402,12 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
           encode_map(&tm.d, delta, s.bf16, W, H, channels, batch, p0.var.cmax, p0.cpw) &&
           encode_map(&tm.b, B, s.bf16, W, H, N, static_cast<long long>(batch) * s.K, p0.var.cmax, nb) &&
           encode_map(&tm.c, C, s.bf16, W, H, N, static_cast<long long>(batch) * s.K, p0.var.cmax, nb);
-    if (!tma) cp = plan_call(s, false);
+    if (!tma) cp = plan_call(s, false, true);
   }
+  // a chain's blocks share distributed shared memory when such a cluster fits on the device
+  if (cp.link == kLinkCluster &&
+      !cluster_fits(tma ? cp.pl.var.fn_tma : cp.pl.var.fn_plain, cp.pl.warps * 32, cp.smem, cp.pl.nseg))
+    cp = plan_call(s, tma, false);
   const Plan& pl = cp.pl;
   const KernelFn fn = tma ? pl.var.fn_tma : pl.var.fn_plain;
 
@@ -360,6 +418,7 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
   prm.n_cgroups = pl.n_cgroups; prm.n_chains = pl.n_chains;
   prm.strips = pl.strips; prm.wpc = pl.wpc; prm.chains_per_block = pl.chains_per_block;
   prm.nseg = pl.nseg;
+  prm.link = cp.link;
   prm.timeout_ns = kTimeoutNs;
   prm.yacc_stride = cp.yacc_stride;
   prm.out_f32 = s.out_f32 ? 1 : 0;
@@ -367,7 +426,7 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
 
   Workspace* ws = nullptr;
   if (cp.need_ws) {
-    if (pl.nseg > 1) {
+    if (cp.link == kLinkGlobal) {
       // a chain's blocks must be able to be resident together (producer back-pressure)
       int per_sm = 0;
       if (!allow_smem(fn, cp.smem)) return SCAN2D_E_LAUNCH;
@@ -377,7 +436,7 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
       }
       if (static_cast<long long>(per_sm) * nsm < pl.nseg) return SCAN2D_E_DIMS;
     }
-    ws = get_workspace(dev, st, cp.items, cp.carry_bytes + cp.yacc_bytes);
+    ws = get_workspace(dev, st, cp.link == kLinkGlobal ? cp.items : 0, cp.carry_bytes + cp.yacc_bytes);
     if (!ws) return SCAN2D_E_NOMEM;
     char* base = static_cast<char*>(ws->ptr);
     const size_t cap = ws->cap_items;
@@ -396,12 +455,13 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
   };
 
   const int threads = pl.warps * 32;
+  const int cluster = cp.link == kLinkCluster ? pl.nseg : 1;
   if (!cp.global_multi) {
     prm.mode = cp.smem_multi ? kSmemMulti : kSingle;
     prm.orient_count = cp.smem_multi ? cp.nk : 1;
     for (int k = 0; k < prm.orient_count; ++k) { prm.orient_code[k] = cp.codes[k]; prm.orient_k[k] = k; }
     prm.gen = next_gen();
-    return launch(fn, threads, prm, tm, cp.smem, cp.grid, st);
+    return launch(fn, threads, prm, tm, cp.smem, cp.grid, cluster, st);
   }
   for (int k = 0; k < cp.nk; ++k) {
     prm.mode = k == 0 ? kGlobalFirst : (k == cp.nk - 1 ? kGlobalLast : kGlobalMid);
@@ -409,7 +469,7 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
     prm.orient_code[0] = cp.codes[k];
     prm.orient_k[0] = k;
     prm.gen = next_gen();
-    rc = launch(fn, threads, prm, tm, cp.smem, cp.grid, st);
+    rc = launch(fn, threads, prm, tm, cp.smem, cp.grid, cluster, st);
     if (rc) return rc;
   }
   return SCAN2D_OK;
@@ -435,11 +495,13 @@ int scan2d_query_plan(int batch, int channels, int H, int W, int N, unsigned fla
   if (!out) return SCAN2D_E_NULL;
   // the layout decides TMA; with 16-byte aligned buffers only the row stride matters
   const bool tma = (static_cast<size_t>(W) * s.in_elem) % 16 == 0;
-  const scan2d::CallPlan cp = scan2d::plan_call(s, tma);
+  // chains of up to 16 blocks are planned as clusters (the call itself falls back to the
+  // global ring if such a cluster cannot be resident on the device)
+  const scan2d::CallPlan cp = scan2d::plan_call(s, tma, true);
   const long long v[SCAN2D_PLAN_FIELDS] = {
       cp.launches, cp.grid, cp.pl.warps * 32, static_cast<long long>(cp.smem), cp.pl.nseg,
       cp.pl.var.cmax, cp.pl.wpc, cp.smem_multi ? 1 : (cp.global_multi ? 2 : 0), cp.pl.var.ng,
-      static_cast<long long>(cp.ws_bytes), cp.pl.var.g, tma ? 1 : 0};
+      static_cast<long long>(cp.ws_bytes), cp.pl.var.g, tma ? 1 : 0, cp.link};
   for (int k = 0; k < n_out && k < SCAN2D_PLAN_FIELDS; ++k) out[k] = v[k];
   return SCAN2D_OK;
 }

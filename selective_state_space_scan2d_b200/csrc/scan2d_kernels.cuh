@@ -13,18 +13,23 @@
 //     behind, by how many values shared memory can hand to the lanes (32 lane-words per
 //     clock).  A lane therefore owns an outer-product block of G channels x NG states:
 //     per position it reads G values of x and delta and NG values of B and C and does
-//     G*NG updates, and the G = 2 channels pair up into packed f32x2 FMAs.
+//     G*NG updates.
 //   * lane = (channel group cg = lane>>2) x (state group q = lane&3); lane q holds states
 //     n = q, q+4, q+8, ...; a warp covers 8*G channels and a strip of CMAX columns.
+//   * Everything but the horizontal recurrence is done on pairs of adjacent columns with
+//     packed f32x2 instructions (adjacent columns are adjacent in shared memory, so the
+//     pairs need no repacking).
 //   * A warp walks all rows of its strip in scan order.  The vertical state of every
 //     (column, channel, state) it owns stays in registers for the whole walk, so the
 //     vertical scan needs no communication.
-//   * The horizontal scan crosses strips.  Inside a block the warps of one chain run
-//     skewed by one row (warp w is on row tau-w at step tau) and hand over the carry
-//     through shared memory; between the blocks of a chain the carry goes through a ring
-//     in global memory with release/acquire flags.  Blocks take (chain, segment) from a
-//     ticket counter, so a block only waits on blocks that started before it, and every
-//     wait is bounded in time.
+//   * The horizontal scan crosses strips.  Warps are not lock-stepped: the carry (the row's
+//     last hh) goes to the next strip's warp through a small shared-memory ring guarded by
+//     full/empty mbarriers.  The blocks of one chain form a thread-block cluster and the
+//     last warp of a block writes straight into the next block's ring (distributed shared
+//     memory, remote mbarrier arrive), so no compute warp ever waits on a global-memory
+//     fence.  Chains longer than a cluster fall back to a ring in global memory with
+//     release/acquire flags (blocks take their place from a ticket counter, so a block only
+//     waits on blocks that started before it).  Every wait is bounded in time.
 //   * Each warp stages the row tiles of its strip (x, delta for its channels, B, C for all
 //     states) into a private shared-memory ring, by TMA (cp.async.bulk.tensor, mbarrier
 //     completion) when the strides allow, else by plain loads prefetched one row ahead.
@@ -46,9 +51,11 @@ namespace scan2d {
 
 constexpr int kQ = 4;                  // state-group lanes per channel group
 constexpr int kGroups = 8;             // channel groups per warp
-constexpr int kRing = 16;              // carry rows buffered between blocks
+constexpr int kRing = 16;              // carry rows buffered in global memory between blocks
+constexpr int kCarryRing = 4;          // carry rows buffered in shared memory between warps
 constexpr int kMaxWarps = 8;           // warps per block
-constexpr int kDepth = 3;              // rows staged ahead per warp (TMA path)
+constexpr int kDepth = 4;              // rows staged ahead per warp (TMA path)
+constexpr int kPublish = 4;            // global fallback: rows per flag release
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum Mode : int {
@@ -57,6 +64,12 @@ enum Mode : int {
   kGlobalFirst = 2,  // first of several launches: yacc = acc + D x
   kGlobalMid = 3,    // yacc += acc
   kGlobalLast = 4,   // y = yacc + acc
+};
+
+enum Link : int {
+  kLinkNone = 0,     // one block per chain
+  kLinkCluster = 1,  // the chain's blocks form a cluster; carries through distributed smem
+  kLinkGlobal = 2,   // carries through a ring in global memory
 };
 
 struct Params {
@@ -75,6 +88,7 @@ struct Params {
   int wpc;                  // warps (strips) per chain inside one block
   int chains_per_block;     // > 1 only when nseg == 1
   int nseg;                 // blocks per chain
+  int link;                 // Link
   int orient_count;         // orientations handled by this launch
   int orient_code[4];       // orientation number (bit0 = flip W, bit1 = flip H)
   int orient_k[4];          // index of the orientation's B_k, C_k
@@ -129,6 +143,23 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+__device__ __forceinline__ unsigned cluster_rank() {
+  unsigned r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// shared::cluster address of the same shared-memory location in block `rank` of the cluster
+__device__ __forceinline__ uint32_t map_rank(uint32_t local, unsigned rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
@@ -137,16 +168,29 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
+__device__ __forceinline__ void mbar_arrive_local(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, unsigned parity) {
   unsigned ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
+}
+
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
 }
 
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar,
@@ -162,8 +206,8 @@ __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Records a device error once and marks this launch generation aborted (every other wait
-// of the launch then gives up at once).
+// Records a device error once and marks this launch generation aborted: every other wait of
+// the launch then gives up at once (checked through ctrl[2] where a ctrl block exists).
 __device__ __noinline__ void report_timeout(unsigned long long* ctrl, unsigned long long gen) {
   atomicCAS(&g_device_error, 0, SCAN2D_E_TIMEOUT);
   if (ctrl != nullptr) st_release(&ctrl[2], gen);
@@ -189,61 +233,42 @@ __device__ __noinline__ bool wait_geq(const unsigned long long* p, unsigned long
   }
 }
 
-// Bounded wait for phase `parity` of a TMA mbarrier.
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, unsigned parity, unsigned long long* ctrl,
-                                       unsigned long long gen, long long timeout_ns) {
+// Bounded wait for phase `parity` of an mbarrier (TMA completion or a carry ring slot).
+// `aborted` (per warp) short-cuts every later wait once one has timed out.
+__device__ __noinline__ void mbar_wait(uint32_t bar, unsigned parity, unsigned long long* ctrl,
+                                       unsigned long long gen, long long timeout_ns, bool& aborted) {
+  if (aborted) return;
   long long t0 = 0;
   for (unsigned it = 0;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return;
     if ((it & 15u) == 0u) {
       const long long now = global_ns();
       if (it == 0u) t0 = now;
       if (now - t0 > timeout_ns || it > (1u << 28)) {
         report_timeout(ctrl, gen);
-        return false;
+        aborted = true;
+        return;
       }
     }
   }
 }
 
-// ---- G-wide vectors: G = 2 channels per lane pair into packed f32x2 instructions --------
-template <int G> struct VecT;
-template <> struct VecT<1> { using T = float; };
-template <> struct VecT<2> { using T = float2; };
-
-__device__ __forceinline__ float vmul(float a, float b) { return a * b; }
-__device__ __forceinline__ float vfma(float a, float b, float c) { return fmaf(a, b, c); }
-__device__ __forceinline__ float vex2(float a) { return ex2_approx(a); }
-__device__ __forceinline__ float vget(float a, int) { return a; }
-
-__device__ __forceinline__ float2 vmul(float2 a, float2 b) { return __fmul2_rn(a, b); }
-__device__ __forceinline__ float2 vfma(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
-__device__ __forceinline__ float2 vex2(float2 a) { return make_float2(ex2_approx(a.x), ex2_approx(a.y)); }
-__device__ __forceinline__ float vget(float2 a, int c) { return c == 0 ? a.x : a.y; }
-
-template <int G> __device__ __forceinline__ typename VecT<G>::T vsplat(float a);
-template <> __device__ __forceinline__ float vsplat<1>(float a) { return a; }
-template <> __device__ __forceinline__ float2 vsplat<2>(float a) { return make_float2(a, a); }
-
-template <int G> __device__ __forceinline__ typename VecT<G>::T vmake(const float* a);
-template <> __device__ __forceinline__ float vmake<1>(const float* a) { return a[0]; }
-template <> __device__ __forceinline__ float2 vmake<2>(const float* a) { return make_float2(a[0], a[1]); }
-
 // ---- staged-row element access ------------------------------------------------------------
-// A 16-byte vector holds 4 fp32 or 8 bf16 values of consecutive columns.
+// A 16-byte vector holds 4 fp32 or 8 bf16 values of consecutive columns; pair(v, p) returns
+// columns 2p and 2p+1 of it as a float2.
 template <typename Tin> struct Elem;
 template <> struct Elem<float> {
   static constexpr int kPerVec = 4;
-  static __device__ __forceinline__ float get(const uint4& v, int j) {
-    const unsigned w = j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
-    return __uint_as_float(w);
+  static __device__ __forceinline__ float2 pair(const uint4& v, int p) {
+    return p == 0 ? make_float2(__uint_as_float(v.x), __uint_as_float(v.y))
+                  : make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
   }
 };
 template <> struct Elem<uint16_t> {
   static constexpr int kPerVec = 8;
-  static __device__ __forceinline__ float get(const uint4& v, int j) {
-    const unsigned w = (j >> 1) == 0 ? v.x : ((j >> 1) == 1 ? v.y : ((j >> 1) == 2 ? v.z : v.w));
-    return __uint_as_float((j & 1) ? (w & 0xffff0000u) : (w << 16));
+  static __device__ __forceinline__ float2 pair(const uint4& v, int p) {
+    const unsigned w = p == 0 ? v.x : (p == 1 ? v.y : (p == 2 ? v.z : v.w));
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
   }
 };
 
@@ -277,7 +302,7 @@ __device__ __forceinline__ void store_out4(void* y, size_t idx, const float* v, 
   else store4(static_cast<uint16_t*>(y) + idx, v);
 }
 
-// ---- shared-memory tile of one strip row ------------------------------------------------------
+// ---- shared memory of one block ---------------------------------------------------------------
 template <typename Tin, int NG, int G, int CMAX>
 struct Layout {
   static constexpr int ESZ = static_cast<int>(sizeof(Tin));
@@ -286,24 +311,36 @@ struct Layout {
   static constexpr int X_BYTES = CPW * CMAX * ESZ;           // [CPW][CMAX]
   static constexpr int B_BYTES = NB * CMAX * ESZ;            // [NB][CMAX]
   static constexpr int r128(int v) { return (v + 127) / 128 * 128; }
-  // every region starts on a 128-byte boundary (TMA destination alignment)
+  // one staged strip row; every region starts on a 128-byte boundary (TMA destinations)
   static constexpr int X_OFF = 0;                                        // element offsets
   static constexpr int D_OFF = r128(X_BYTES) / ESZ;
   static constexpr int B_OFF = D_OFF + r128(X_BYTES) / ESZ;
   static constexpr int C_OFF = B_OFF + r128(B_BYTES) / ESZ;
-  static constexpr int BYTES = (C_OFF * ESZ) + r128(B_BYTES);
+  static constexpr int TILE_BYTES = (C_OFF * ESZ) + r128(B_BYTES);
   static constexpr int TX_BYTES = 2 * X_BYTES + 2 * B_BYTES;
   static constexpr int DENSE = (2 * CPW + 2 * NB) * CMAX;    // tile values without padding
-  static constexpr int E = CMAX * G;                         // partial outputs per lane per row
   static constexpr int PLAIN_PER_LANE = DENSE / 32;          // plain-load path: values per lane
+  static constexpr int CARRY = G * NG;                       // carry floats per lane
+  static constexpr int CARRY_PAD = (CARRY + 3) / 4 * 4;      // ... padded to whole float4s
+  static constexpr int CARRY_SLOT_BYTES = 32 * CARRY_PAD * 4;  // one carry row of a warp
+  static constexpr int E = CMAX * G;                         // partial outputs per lane per row
+  static constexpr int NP = CMAX / 2;                        // column pairs per strip
 };
+
+// Dynamic shared memory, in this order (all offsets multiples of 128 bytes):
+//   carry rings   [warps][kCarryRing] carry rows          (incoming carries of each warp)
+//   tile rings    [warps][depth] staged strip rows
+//   accumulator   [chains_per_block][CPW][yacc_stride] floats (kSmemMulti only)
+template <typename Tin, int NG, int G, int CMAX>
+__host__ __device__ constexpr size_t carry_ring_bytes(int warps) {
+  return static_cast<size_t>(warps) * kCarryRing * Layout<Tin, NG, G, CMAX>::CARRY_SLOT_BYTES;
+}
 
 // ---- the kernel ------------------------------------------------------------------------------
 template <typename Tin, int NG, int G, int CMAX, bool TMA>
 __global__ void __launch_bounds__(kMaxWarps * 32)
 scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps tm) {
   using L = Layout<Tin, NG, G, CMAX>;
-  using V = typename VecT<G>::T;
   constexpr int PV = Elem<Tin>::kPerVec;
   static_assert(CMAX % PV == 0, "strip width must hold whole 16-byte vectors");
   static_assert(L::E % 4 == 0, "reduce-scatter needs 4 | CMAX*G");
@@ -311,22 +348,31 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   constexpr int DEPTH = TMA ? kDepth : 1;
   constexpr int NVEC = CMAX / PV;                            // 16-byte vectors per strip row
   constexpr int E = L::E;
+  constexpr int NP = L::NP;
 
   extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ uint64_t s_bar[kMaxWarps][kDepth];
+  __shared__ uint64_t s_tma_bar[kMaxWarps][kDepth];
+  __shared__ uint64_t s_full[kMaxWarps][kCarryRing];         // carry slot written (consumer side)
+  __shared__ uint64_t s_empty[kMaxWarps][kCarryRing];        // carry slot read (producer side)
   __shared__ int s_item;
 
   const unsigned FULL = 0xffffffffu;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
   const int slot = warp / p.wpc;            // chain slot inside the block
   const int w = warp - slot * p.wpc;        // strip inside the segment
   const int cg = lane >> 2;                 // channel group
   const int q = lane & 3;                   // state group
+  const bool cluster = p.link == kLinkCluster;
+  const bool global_link = p.link == kLinkGlobal;
 
   // ---- which chain and segment -------------------------------------------------------
   int chain, seg;
-  if (p.nseg > 1) {
+  if (cluster) {
+    seg = static_cast<int>(cluster_rank());
+    chain = blockIdx.x / p.nseg;
+  } else if (global_link) {
     if (threadIdx.x == 0) s_item = static_cast<int>(atomicAdd(&p.ctrl[0], 1ull));
     __syncthreads();
     chain = s_item / p.nseg;
@@ -340,54 +386,57 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   const int grp = chain_ok ? chain - b * p.n_cgroups : 0;
   const int u_scan = seg * p.wpc + w;                        // strip position in scan order
   const bool strip_ok = chain_ok && u_scan < p.strips;       // warp-uniform
+  // does the next strip of the chain exist (and who owns it)?
+  const bool next_local = strip_ok && w < p.wpc - 1 && u_scan + 1 < p.strips;
+  const bool next_remote = strip_ok && w == p.wpc - 1 && seg < p.nseg - 1 && u_scan + 1 < p.strips;
+  const bool has_left = strip_ok && u_scan > 0;              // a carry comes in
+  const bool left_global = has_left && w == 0 && global_link;
+  const bool left_remote = has_left && w == 0 && cluster;    // carry comes from the previous block
 
   const int H = p.H, W = p.W, N = p.N;
   const size_t HW = static_cast<size_t>(H) * W;
   const int ch0 = grp * L::CPW + cg * G;                     // first channel of this lane
 
-  // per-lane constants: A * log2(e) per (channel, state), Dskip per channel
-  V A2[NG];
-  V Dd;
-  {
-    float dd[G];
+  // per-lane constants: A * log2(e) per (channel, state) as a splat pair, Dskip per channel
+  float2 A2[G][NG];
+  float2 Dd[G];
 #pragma unroll
-    for (int c = 0; c < G; ++c) {
-      const int d = ch0 + c;
-      dd[c] = (chain_ok && d < p.channels && p.Dskip != nullptr) ? __ldg(p.Dskip + d) : 0.f;
-    }
-    Dd = vmake<G>(dd);
+  for (int c = 0; c < G; ++c) {
+    const int d = ch0 + c;
+    const bool dok = chain_ok && d < p.channels;
+    const float dv = (dok && p.Dskip != nullptr) ? __ldg(p.Dskip + d) : 0.f;
+    Dd[c] = make_float2(dv, dv);
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
-      float a[G];
       const int n = q + kQ * g;
-#pragma unroll
-      for (int c = 0; c < G; ++c) {
-        const int d = ch0 + c;
-        a[c] = (chain_ok && d < p.channels && n < N) ? __ldg(p.A + static_cast<size_t>(d) * N + n) * kLog2e : 0.f;
-      }
-      A2[g] = vmake<G>(a);
+      const float a = (dok && n < N) ? __ldg(p.A + static_cast<size_t>(d) * N + n) * kLog2e : 0.f;
+      A2[c][g] = make_float2(a, a);
     }
   }
 
-  // ---- shared memory: carries | staged rows | output accumulator ----------------------------
-  const int carry_floats = p.wpc > 1 ? 2 * kMaxWarps * 32 * G * NG : 0;
-  float* carry_s = reinterpret_cast<float*>(smem);
-  unsigned char* slots = smem + carry_floats * sizeof(float) + warp * DEPTH * L::BYTES;
-  float* yacc_s = reinterpret_cast<float*>(smem + carry_floats * sizeof(float) +
-                                           (p.wpc * p.chains_per_block) * DEPTH * L::BYTES);
+  // ---- shared memory ---------------------------------------------------------------------
+  unsigned char* carry_base = smem;
+  unsigned char* tiles = smem + carry_ring_bytes<Tin, NG, G, CMAX>(nwarps) + warp * DEPTH * L::TILE_BYTES;
+  float* yacc_s = reinterpret_cast<float*>(smem + carry_ring_bytes<Tin, NG, G, CMAX>(nwarps) +
+                                           static_cast<size_t>(nwarps) * DEPTH * L::TILE_BYTES);
+  auto carry_slot = [&](int wr, int s) -> float* {
+    return reinterpret_cast<float*>(carry_base + (wr * kCarryRing + s) * L::CARRY_SLOT_BYTES);
+  };
 
-  if (TMA) {
-    if (lane == 0) {
+  if (lane == 0) {
 #pragma unroll
-      for (int s = 0; s < DEPTH; ++s) mbar_init(&s_bar[warp][s], 1);
-      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    for (int s = 0; s < DEPTH; ++s) mbar_init(&s_tma_bar[warp][s], 1);
+#pragma unroll
+    for (int s = 0; s < kCarryRing; ++s) {
+      mbar_init(&s_full[warp][s], 32);
+      mbar_init(&s_empty[warp][s], 32);
     }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  __syncthreads();
+  if (cluster) cluster_sync();      // every block's barriers exist before any remote arrive
+  else __syncthreads();
 
   const int item = chain * p.nseg + seg;
-  const bool consumer = (w == 0) && seg > 0;
-  const bool producer = (w == p.wpc - 1) && seg < p.nseg - 1;
   const int U = p.orient_count * H;                          // rows this warp walks
 
   // row u of the walk -> (orientation index, stored row, stored strip)
@@ -404,8 +453,8 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
     row_coords(uu, oi, i, t);
     const int k = p.orient_k[oi];
     const int s = uu % DEPTH;
-    unsigned char* dst = slots + s * L::BYTES;
-    uint64_t* bar = &s_bar[warp][s];
+    unsigned char* dst = tiles + s * L::TILE_BYTES;
+    uint64_t* bar = &s_tma_bar[warp][s];
     mbar_expect_tx(bar, L::TX_BYTES);
     tma_load_4d(dst + L::X_OFF * L::ESZ, &tm.x, bar, t * CMAX, i, grp * L::CPW, b);
     tma_load_4d(dst + L::D_OFF * L::ESZ, &tm.d, bar, t * CMAX, i, grp * L::CPW, b);
@@ -413,8 +462,8 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
     tma_load_4d(dst + L::C_OFF * L::ESZ, &tm.c, bar, t * CMAX, i, 0, b * p.K + k);
   };
 
-  // plain-load path: this lane's share of row u's tile, zero outside the tensors.  Value
-  // e of the dense tile goes to tile offset plain_dst(e).
+  // plain-load path: this lane's share of row u's tile, zero outside the tensors.  Value e
+  // of the dense tile goes to tile offset plain_dst(e).
   auto plain_split = [&](int e, int& region, int& rr, int& cc) {
     if (e < 2 * L::CPW * CMAX) {
       region = e / (L::CPW * CMAX);
@@ -459,6 +508,7 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
     }
   };
 
+  bool aborted = false;
   if (strip_ok) {
     if (TMA) {
       if (lane == 0)
@@ -466,6 +516,18 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
     } else {
       plain_load(0);
     }
+  }
+
+  // where this warp's carries go: the next warp of this block, or warp 0 of the next block
+  const uint32_t next_full0 = smem_u32(&s_full[next_local ? warp + 1 : 0][0]);
+  const uint32_t my_empty0 = smem_u32(&s_empty[warp][0]);
+  uint32_t next_ring_cl = 0, next_full_cl = 0, prev_empty_cl = 0;
+  if (cluster) {
+    if (next_remote) {
+      next_ring_cl = map_rank(smem_u32(carry_slot(0, 0)), seg + 1);
+      next_full_cl = map_rank(smem_u32(&s_full[0][0]), seg + 1);
+    }
+    if (left_remote) prev_empty_cl = map_rank(smem_u32(&s_empty[p.wpc - 1][0]), seg - 1);
   }
 
   int u = 0;                                                 // rows of the walk done so far
@@ -476,200 +538,251 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
     const int col0 = t * CMAX;
     const bool add_dx = (p.mode == kSingle || p.mode == kGlobalFirst || (p.mode == kSmemMulti && oi == 0));
 
-    V v[CMAX][NG];
+    float2 v[NP][G][NG];                                     // vertical state, column pairs
 #pragma unroll
-    for (int j = 0; j < CMAX; ++j)
+    for (int pp = 0; pp < NP; ++pp)
 #pragma unroll
-      for (int g = 0; g < NG; ++g) v[j][g] = vsplat<G>(0.f);
+      for (int c = 0; c < G; ++c)
+#pragma unroll
+        for (int g = 0; g < NG; ++g) v[pp][c][g] = make_float2(0.f, 0.f);
 
-    const int steps = H + p.wpc - 1;
-    for (int tau = 0; tau < steps; ++tau) {
-      const int r = tau - w;
-      const bool active = strip_ok && r >= 0 && r < H;      // warp-uniform
-      if (active) {
-        const int i = flipH ? H - 1 - r : r;
-        const int s = u % DEPTH;
-        const Tin* tile = reinterpret_cast<const Tin*>(slots + s * L::BYTES);
+    for (int r = 0; r < H && strip_ok; ++r, ++u) {
+      const int i = flipH ? H - 1 - r : r;
+      const int s = u % DEPTH;
+      const Tin* tile = reinterpret_cast<const Tin*>(tiles + s * L::TILE_BYTES);
+      const int cs = u % kCarryRing;                         // carry ring slot of this row
+      const unsigned cpar = static_cast<unsigned>((u / kCarryRing) & 1);
 
-        // ---- (1) this row's tile is in shared memory -----------------------------------
-        if (TMA) {
-          mbar_wait(&s_bar[warp][s], static_cast<unsigned>((u / DEPTH) & 1), p.ctrl, p.gen, p.timeout_ns);
-        } else {
-          Tin* dst = reinterpret_cast<Tin*>(slots);
+      // ---- (1) this row's tile is in shared memory -----------------------------------
+      if (TMA) {
+        mbar_wait(smem_u32(&s_tma_bar[warp][s]), static_cast<unsigned>((u / DEPTH) & 1), p.ctrl, p.gen,
+                  p.timeout_ns, aborted);
+      } else {
+        Tin* dst = reinterpret_cast<Tin*>(tiles);
 #pragma unroll
-          for (int m = 0; m < L::PLAIN_PER_LANE; ++m) dst[plain_dst(lane + 32 * m)] = pre[m];
-          __syncwarp();
-          if (u + 1 < U) plain_load(u + 1);
-        }
-
-        // ---- (2) carry-in: hh at the column before this strip (scan order) ----------------
-        V hh[NG];
-        if (w > 0) {
-          const float* src = carry_s + (((tau - 1) & 1) * kMaxWarps + (warp - 1)) * 32 * G * NG + lane * G * NG;
-#pragma unroll
-          for (int g = 0; g < NG; ++g) hh[g] = vmake<G>(src + g * G);
-        } else if (consumer) {
-          const unsigned long long want = tag(p.gen, r + 1);
-          if (lane == 0) wait_geq(&p.flags[item - 1], want, p.ctrl, p.gen, p.timeout_ns);
-          __syncwarp();
-          const bool ok = ld_acquire(&p.flags[item - 1]) >= want;   // every lane acquires
-          const float* src = p.carry + ((static_cast<size_t>(item - 1) * kRing + (r % kRing)) * 32 + lane) * G * NG;
-#pragma unroll
-          for (int g = 0; g < NG; ++g) {
-            float tmp[G];
-#pragma unroll
-            for (int c = 0; c < G; ++c) tmp[c] = ok ? __ldcg(src + g * G + c) : 0.f;
-            hh[g] = vmake<G>(tmp);
-          }
-        } else {
-#pragma unroll
-          for (int g = 0; g < NG; ++g) hh[g] = vsplat<G>(0.f);
-        }
-
-        // ---- (3) the strip's columns of this row ------------------------------------------
-        // per lane: G channels (x, delta) and NG states (B, C) of every column, 16-byte vectors
-        V acc[CMAX];
-        auto column = [&](int j, const uint4* xv, const uint4* dv, const uint4* bv, const uint4* cv, int jv) {
-          float xs[G], ds[G];
-#pragma unroll
-          for (int c = 0; c < G; ++c) {
-            xs[c] = Elem<Tin>::get(xv[c], jv);
-            ds[c] = Elem<Tin>::get(dv[c], jv);
-          }
-          const V x2 = vmake<G>(xs);
-          const V d2 = vmake<G>(ds);
-          const V dx = vmul(d2, x2);
-          V a_acc = (add_dx && q == 0) ? vmul(Dd, x2) : vsplat<G>(0.f);
-#pragma unroll
-          for (int g = 0; g < NG; ++g) {
-            const V a = vex2(vmul(d2, A2[g]));
-            const V uu = vmul(dx, vsplat<G>(Elem<Tin>::get(bv[g], jv)));
-            hh[g] = vfma(a, hh[g], uu);
-            v[j][g] = vfma(a, v[j][g], hh[g]);
-            a_acc = vfma(vsplat<G>(Elem<Tin>::get(cv[g], jv)), v[j][g], a_acc);
-          }
-          acc[j] = a_acc;
-        };
-        auto vector_group = [&](int vg, bool rev) {
-          uint4 xv[G], dv[G], bv[NG], cv[NG];
-#pragma unroll
-          for (int c = 0; c < G; ++c) {
-            xv[c] = *reinterpret_cast<const uint4*>(tile + L::X_OFF + (cg * G + c) * CMAX + vg * PV);
-            dv[c] = *reinterpret_cast<const uint4*>(tile + L::D_OFF + (cg * G + c) * CMAX + vg * PV);
-          }
-#pragma unroll
-          for (int g = 0; g < NG; ++g) {
-            bv[g] = *reinterpret_cast<const uint4*>(tile + L::B_OFF + (q + kQ * g) * CMAX + vg * PV);
-            cv[g] = *reinterpret_cast<const uint4*>(tile + L::C_OFF + (q + kQ * g) * CMAX + vg * PV);
-          }
-          if (!rev) {
-#pragma unroll
-            for (int jv = 0; jv < PV; ++jv) column(vg * PV + jv, xv, dv, bv, cv, jv);
-          } else {
-#pragma unroll
-            for (int jv = PV - 1; jv >= 0; --jv) column(vg * PV + jv, xv, dv, bv, cv, jv);
-          }
-        };
-        if (!flipW) {
-#pragma unroll
-          for (int vg = 0; vg < NVEC; ++vg) vector_group(vg, false);
-        } else {
-#pragma unroll
-          for (int vg = NVEC - 1; vg >= 0; --vg) vector_group(vg, true);
-        }
-
-        // ---- (4) the tile slot is free again: stage row u + DEPTH into it ---------------------
+        for (int m = 0; m < L::PLAIN_PER_LANE; ++m) dst[plain_dst(lane + 32 * m)] = pre[m];
         __syncwarp();
-        if (TMA && lane == 0 && u + DEPTH < U) {
-          fence_proxy_async();
-          issue_tma(u + DEPTH);
-        }
+        if (u + 1 < U) plain_load(u + 1);
+      }
 
-        // ---- (5) carry-out --------------------------------------------------------------------
-        if (w < p.wpc - 1) {
-          float* dst = carry_s + ((tau & 1) * kMaxWarps + warp) * 32 * G * NG + lane * G * NG;
+      // ---- (2) carry-in: hh at the column before this strip (scan order) ----------------
+      float hh[G][NG];
+      if (left_global) {
+        const unsigned long long want = tag(p.gen, r + 1);
+        if (lane == 0) wait_geq(&p.flags[item - 1], want, p.ctrl, p.gen, p.timeout_ns);
+        __syncwarp();
+        const bool ok = ld_acquire(&p.flags[item - 1]) >= want;   // every lane acquires
+        const float* src = p.carry + ((static_cast<size_t>(item - 1) * kRing + (r % kRing)) * 32 + lane) * L::CARRY;
 #pragma unroll
-          for (int g = 0; g < NG; ++g)
+        for (int c = 0; c < G; ++c)
 #pragma unroll
-            for (int c = 0; c < G; ++c) dst[g * G + c] = vget(hh[g], c);
-        } else if (producer) {
-          if (r >= kRing) {
-            const unsigned long long want = tag(p.gen, r - kRing + 1);
-            if (lane == 0) wait_geq(&p.acks[item + 1], want, p.ctrl, p.gen, p.timeout_ns);
-            __syncwarp();
-            (void)ld_acquire(&p.acks[item + 1]);           // orders this lane's ring writes
+          for (int g = 0; g < NG; ++g) hh[c][g] = ok ? __ldcg(src + c * NG + g) : 0.f;
+      } else if (has_left) {
+        mbar_wait(smem_u32(&s_full[warp][cs]), cpar, p.ctrl, p.gen, p.timeout_ns, aborted);
+        const float4* src = reinterpret_cast<const float4*>(carry_slot(warp, cs)) + lane * (L::CARRY_PAD / 4);
+        float in[L::CARRY_PAD];
+#pragma unroll
+        for (int k4 = 0; k4 < L::CARRY_PAD / 4; ++k4) {
+          const float4 f = src[k4];
+          in[4 * k4] = f.x;
+          in[4 * k4 + 1] = f.y;
+          in[4 * k4 + 2] = f.z;
+          in[4 * k4 + 3] = f.w;
+        }
+#pragma unroll
+        for (int c = 0; c < G; ++c)
+#pragma unroll
+          for (int g = 0; g < NG; ++g) hh[c][g] = in[c * NG + g];
+        // free the slot: the producer waits on its own empty barrier
+        if (left_remote) mbar_arrive_remote(prev_empty_cl + cs * 8);
+        else mbar_arrive_local(smem_u32(&s_empty[warp - 1][cs]));
+      } else {
+#pragma unroll
+        for (int c = 0; c < G; ++c)
+#pragma unroll
+          for (int g = 0; g < NG; ++g) hh[c][g] = 0.f;
+      }
+
+      // ---- (3) the strip's columns of this row, two adjacent columns at a time -------------
+      float2 acc[NP][G];
+      auto vec_group = [&](int vg, bool rev) {
+        uint4 xv[G], dv[G], bv[NG], cv[NG];
+#pragma unroll
+        for (int c = 0; c < G; ++c) {
+          xv[c] = *reinterpret_cast<const uint4*>(tile + L::X_OFF + (cg * G + c) * CMAX + vg * PV);
+          dv[c] = *reinterpret_cast<const uint4*>(tile + L::D_OFF + (cg * G + c) * CMAX + vg * PV);
+        }
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+          bv[g] = *reinterpret_cast<const uint4*>(tile + L::B_OFF + (q + kQ * g) * CMAX + vg * PV);
+          cv[g] = *reinterpret_cast<const uint4*>(tile + L::C_OFF + (q + kQ * g) * CMAX + vg * PV);
+        }
+#pragma unroll
+        for (int k = 0; k < PV / 2; ++k) {
+          const int kp = rev ? PV / 2 - 1 - k : k;           // pair inside the vector
+          const int pp = vg * (PV / 2) + kp;                 // pair inside the strip
+#pragma unroll
+          for (int c = 0; c < G; ++c) {
+            const float2 x2 = Elem<Tin>::pair(xv[c], kp);
+            const float2 d2 = Elem<Tin>::pair(dv[c], kp);
+            const float2 dx = __fmul2_rn(d2, x2);
+            float2 a_acc = (add_dx && q == 0) ? __fmul2_rn(Dd[c], x2) : make_float2(0.f, 0.f);
+#pragma unroll
+            for (int g = 0; g < NG; ++g) {
+              const float2 arg = __fmul2_rn(d2, A2[c][g]);
+              const float2 a = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+              const float2 uu = __fmul2_rn(dx, Elem<Tin>::pair(bv[g], kp));
+              float2 h2;
+              if (!rev) {
+                h2.x = fmaf(a.x, hh[c][g], uu.x);
+                h2.y = fmaf(a.y, h2.x, uu.y);
+                hh[c][g] = h2.y;
+              } else {
+                h2.y = fmaf(a.y, hh[c][g], uu.y);
+                h2.x = fmaf(a.x, h2.y, uu.x);
+                hh[c][g] = h2.x;
+              }
+              v[pp][c][g] = __ffma2_rn(a, v[pp][c][g], h2);
+              a_acc = __ffma2_rn(Elem<Tin>::pair(cv[g], kp), v[pp][c][g], a_acc);
+            }
+            acc[pp][c] = a_acc;
           }
-          float* dst = p.carry + ((static_cast<size_t>(item) * kRing + (r % kRing)) * 32 + lane) * G * NG;
+        }
+      };
+      if (!flipW) {
 #pragma unroll
-          for (int g = 0; g < NG; ++g)
+        for (int vg = 0; vg < NVEC; ++vg) vec_group(vg, false);
+      } else {
 #pragma unroll
-            for (int c = 0; c < G; ++c) __stcg(dst + g * G + c, vget(hh[g], c));
+        for (int vg = NVEC - 1; vg >= 0; --vg) vec_group(vg, true);
+      }
+
+      // ---- (4) the tile slot is free again: stage row u + DEPTH into it ---------------------
+      __syncwarp();
+      if (TMA && lane == 0 && u + DEPTH < U) {
+        fence_proxy_async();
+        issue_tma(u + DEPTH);
+      }
+
+      // ---- (5) carry-out to the next strip ---------------------------------------------------
+      if (next_local || (next_remote && cluster)) {
+        // the slot is free once the consumer released its previous use
+        if (u >= kCarryRing)
+          mbar_wait(my_empty0 + cs * 8, cpar ^ 1u, p.ctrl, p.gen, p.timeout_ns, aborted);
+        float out[L::CARRY_PAD];
+#pragma unroll
+        for (int e = L::CARRY; e < L::CARRY_PAD; ++e) out[e] = 0.f;
+#pragma unroll
+        for (int c = 0; c < G; ++c)
+#pragma unroll
+          for (int g = 0; g < NG; ++g) out[c * NG + g] = hh[c][g];
+        if (next_local) {
+          float4* dst = reinterpret_cast<float4*>(carry_slot(warp + 1, cs)) + lane * (L::CARRY_PAD / 4);
+#pragma unroll
+          for (int k4 = 0; k4 < L::CARRY_PAD / 4; ++k4)
+            dst[k4] = make_float4(out[4 * k4], out[4 * k4 + 1], out[4 * k4 + 2], out[4 * k4 + 3]);
+          mbar_arrive_local(next_full0 + cs * 8);
+        } else {
+          const uint32_t dst = next_ring_cl + cs * L::CARRY_SLOT_BYTES + lane * L::CARRY_PAD * 4;
+#pragma unroll
+          for (int k4 = 0; k4 < L::CARRY_PAD / 4; ++k4)
+            st_cluster_v4(dst + 16 * k4, out[4 * k4], out[4 * k4 + 1], out[4 * k4 + 2], out[4 * k4 + 3]);
+          mbar_arrive_remote(next_full_cl + cs * 8);
+        }
+      } else if (next_remote && global_link) {
+        if (r >= kRing && (r % kPublish) == 0) {
+          // rows up to r - kRing must have been consumed before their slots are reused
+          const unsigned long long want = tag(p.gen, r - kRing + kPublish);
+          if (lane == 0) wait_geq(&p.acks[item + 1], want, p.ctrl, p.gen, p.timeout_ns);
+          __syncwarp();
+          (void)ld_acquire(&p.acks[item + 1]);           // orders this lane's ring writes
+        }
+        float* dst = p.carry + ((static_cast<size_t>(item) * kRing + (r % kRing)) * 32 + lane) * L::CARRY;
+#pragma unroll
+        for (int c = 0; c < G; ++c)
+#pragma unroll
+          for (int g = 0; g < NG; ++g) __stcg(dst + c * NG + g, hh[c][g]);
+        if ((r + 1) % kPublish == 0 || r == H - 1) {
           __threadfence();
           __syncwarp();
           if (lane == 0) st_release(&p.flags[item], tag(p.gen, r + 1));
         }
-        if (consumer) st_release(&p.acks[item], tag(p.gen, r + 1));   // every lane: its loads are done
+      }
+      if (left_global && ((r + 1) % kPublish == 0 || r == H - 1))
+        st_release(&p.acks[item], tag(p.gen, r + 1));   // every lane: its loads are done
 
-        // ---- (6) reduce over the 4 state groups; lane q keeps the q-th quarter ------------------
-        // flat index e = c*CMAX + j (channel-major)
-        float flat[E];
+      // ---- (6) reduce over the 4 state groups; lane q keeps the q-th quarter ------------------
+      // flat index e = c*CMAX + j (channel-major, j = stored column in the strip)
+      float flat[E];
 #pragma unroll
-        for (int c = 0; c < G; ++c)
+      for (int c = 0; c < G; ++c)
 #pragma unroll
-          for (int j = 0; j < CMAX; ++j) flat[c * CMAX + j] = vget(acc[j], c);
-        float r1[E / 2];
-        const bool hi2 = (q & 2) != 0, hi1 = (q & 1) != 0;
-#pragma unroll
-        for (int e = 0; e < E / 2; ++e) {
-          const float lo = flat[e], hi = flat[e + E / 2];
-          r1[e] = (hi2 ? hi : lo) + __shfl_xor_sync(FULL, hi2 ? lo : hi, 2);
+        for (int pp = 0; pp < NP; ++pp) {
+          flat[c * CMAX + 2 * pp] = acc[pp][c].x;
+          flat[c * CMAX + 2 * pp + 1] = acc[pp][c].y;
         }
-        float own[E / 4];
+      float r1[E / 2];
+      const bool hi2 = (q & 2) != 0, hi1 = (q & 1) != 0;
 #pragma unroll
-        for (int e = 0; e < E / 4; ++e) {
-          const float lo = r1[e], hi = r1[e + E / 4];
-          own[e] = (hi1 ? hi : lo) + __shfl_xor_sync(FULL, hi1 ? lo : hi, 1);
-        }
+      for (int e = 0; e < E / 2; ++e) {
+        const float lo = flat[e], hi = flat[e + E / 2];
+        r1[e] = (hi2 ? hi : lo) + __shfl_xor_sync(FULL, hi2 ? lo : hi, 2);
+      }
+      float own[E / 4];
+#pragma unroll
+      for (int e = 0; e < E / 4; ++e) {
+        const float lo = r1[e], hi = r1[e + E / 4];
+        own[e] = (hi1 ? hi : lo) + __shfl_xor_sync(FULL, hi1 ? lo : hi, 1);
+      }
 
-        // ---- (7) output: channel c, columns j0 .. j0 + E/4 - 1 of the strip --------------------
-        {
-          const int e0 = q * (E / 4);
-          const int c = e0 / CMAX;
-          const int j0 = e0 - c * CMAX;
-          const int d = ch0 + c;
-          if (chain_ok && d < p.channels) {
-            const size_t rowoff = (static_cast<size_t>(b) * p.channels + d) * HW + static_cast<size_t>(i) * W;
-            const int gc = col0 + j0;
-            if (p.mode == kSingle) {
-              if ((E / 4) % 4 == 0 && p.vec_store && gc + E / 4 <= W) {
+      // ---- (7) output: channel c, columns j0 .. j0 + E/4 - 1 of the strip --------------------
+      {
+        const int e0 = q * (E / 4);
+        const int c = e0 / CMAX;
+        const int j0 = e0 - c * CMAX;
+        const int d = ch0 + c;
+        if (d < p.channels) {
+          const size_t rowoff = (static_cast<size_t>(b) * p.channels + d) * HW + static_cast<size_t>(i) * W;
+          const int gc = col0 + j0;
+          if (p.mode == kSingle) {
+            if ((E / 4) % 4 == 0 && p.vec_store && gc + E / 4 <= W) {
 #pragma unroll
-                for (int m = 0; m < E / 4; m += 4) store_out4(p.y, rowoff + gc + m, own + m, p.out_f32);
-              } else {
-#pragma unroll
-                for (int m = 0; m < E / 4; ++m)
-                  if (gc + m < W) store_out(p.y, rowoff + gc + m, own[m], p.out_f32);
-              }
-            } else if (p.mode == kSmemMulti) {
-              float* a = yacc_s + (slot * L::CPW + cg * G + c) * p.yacc_stride + i * W + gc;
-#pragma unroll
-              for (int m = 0; m < E / 4; ++m)
-                if (gc + m < W) a[m] = (oi == 0) ? own[m] : a[m] + own[m];
+              for (int m = 0; m < E / 4; m += 4) store_out4(p.y, rowoff + gc + m, own + m, p.out_f32);
             } else {
 #pragma unroll
-              for (int m = 0; m < E / 4; ++m) {
-                if (gc + m >= W) continue;
-                const size_t idx = rowoff + gc + m;
-                if (p.mode == kGlobalFirst) p.yacc[idx] = own[m];
-                else if (p.mode == kGlobalMid) p.yacc[idx] += own[m];
-                else store_out(p.y, idx, p.yacc[idx] + own[m], p.out_f32);
-              }
+              for (int m = 0; m < E / 4; ++m)
+                if (gc + m < W) store_out(p.y, rowoff + gc + m, own[m], p.out_f32);
+            }
+          } else if (p.mode == kSmemMulti) {
+            float* a = yacc_s + (slot * L::CPW + cg * G + c) * p.yacc_stride + i * W + gc;
+#pragma unroll
+            for (int m = 0; m < E / 4; ++m)
+              if (gc + m < W) a[m] = (oi == 0) ? own[m] : a[m] + own[m];
+          } else {
+#pragma unroll
+            for (int m = 0; m < E / 4; ++m) {
+              if (gc + m >= W) continue;
+              const size_t idx = rowoff + gc + m;
+              if (p.mode == kGlobalFirst) p.yacc[idx] = own[m];
+              else if (p.mode == kGlobalMid) p.yacc[idx] += own[m];
+              else store_out(p.y, idx, p.yacc[idx] + own[m], p.out_f32);
             }
           }
         }
-        ++u;
       }
-      __syncthreads();
     }
+    // orientations summed in shared memory: no warp may start the next orientation (whose
+    // strips map to other columns) before every warp has finished this one
+    if (p.mode == kSmemMulti) __syncthreads();
+  }
+
+  // ---- after a timed-out wait: let this warp's TMA copies still in flight land (bounded) ------
+  if (TMA && aborted && strip_ok && lane == 0) {
+    const int issued = U < u + DEPTH ? U : u + DEPTH;      // rows whose copies were started
+    bool drain_gave_up = false;
+    for (int uu = issued - DEPTH < 0 ? 0 : issued - DEPTH; uu < issued; ++uu)
+      mbar_wait(smem_u32(&s_tma_bar[warp][uu % DEPTH]), static_cast<unsigned>((uu / DEPTH) & 1), p.ctrl,
+                p.gen, p.timeout_ns, drain_gave_up);
   }
 
   // ---- kSmemMulti: write the accumulated maps of this block's chains --------------------------
@@ -685,8 +798,11 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
     }
   }
 
+  // ---- leave together: a cluster's shared memory must outlive the remote arrives into it ----
+  if (cluster) cluster_sync();
+
   // ---- the last block of a ticketed launch resets the counters for the next launch ----------
-  if (p.nseg > 1) {
+  if (global_link) {
     __syncthreads();
     if (threadIdx.x == 0) {
       __threadfence();

@@ -144,7 +144,7 @@ def scan2d_fwd(x, delta, A, B, C, Dskip=None, y=None, flags=None, stream=None):
 
 
 PLAN_FIELDS = ("launches", "grid", "threads", "smem", "nseg", "cols", "wpc", "mode", "ng",
-               "workspace", "g", "tma")
+               "workspace", "g", "tma", "link")
 
 
 def scan2d_query_plan(batch, channels, H, W, N, flags) -> dict:

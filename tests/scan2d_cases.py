@@ -7,6 +7,7 @@ CASES = {
     "f32_two_blocks": ("tiny", dict(batch=1, channels=9, N=16, H=21, W=200)),
     "f32_long_chain_backpressure": ("tiny", dict(batch=1, channels=8, N=16, H=40, W=1030)),
     "f32_long_chain_backpressure_tma": ("tiny", dict(batch=1, channels=16, N=16, H=40, W=1024)),
+    "f32_global_ring_tma": ("tiny", dict(batch=1, channels=16, N=16, H=37, W=1056)),
     "bf16_k1_tma": ("small", dict(batch=2, channels=20, H=9, W=48)),
     "bf16_N4_tma": ("small", dict(batch=1, channels=8, N=4, H=5, W=16)),
     "bf16_14x14": ("small", dict(batch=3, channels=19, H=14, W=14)),

@@ -31,10 +31,17 @@ def test_every_path_is_exercised(plans):
     assert {p["g"] for p in ps} == {1, 2}, "one and two channels per lane"
     assert any(p["wpc"] > 1 and p["nseg"] == 1 for p in ps), "several strips in one block"
     assert any(p["tma"] == 1 and p["mode"] == 0 and p["g"] == 2 for p in ps)
+    assert any(p["link"] == 1 and p["tma"] == 1 for p in ps), "cluster-linked chain, TMA"
+    assert any(p["link"] == 1 and p["tma"] == 0 for p in ps), "cluster-linked chain, plain"
+    assert any(p["link"] == 2 and p["tma"] == 1 for p in ps), "global-ring chain, TMA"
+    assert any(p["link"] == 2 and p["tma"] == 0 for p in ps), "global-ring chain, plain"
+    assert any(p["link"] == 1 and p["nseg"] == 16 for p in ps), "the largest cluster"
 
 
 def test_long_chain_hits_ring_back_pressure(plans):
     # 40 rows > the 16-row carry ring, 9+ segments: producers must wait for consumers
-    for case in ("f32_long_chain_backpressure", "f32_long_chain_backpressure_tma"):
-        assert plans[case]["nseg"] >= 8
-    assert plans["f32_long_chain_backpressure_tma"]["tma"] == 1
+    # 37-40 rows > the 16-row global ring and the 4-row shared-memory ring
+    for case in ("f32_long_chain_backpressure", "f32_global_ring_tma"):
+        assert plans[case]["link"] == 2 and plans[case]["nseg"] > 16
+    assert plans["f32_global_ring_tma"]["tma"] == 1
+    assert plans["f32_long_chain_backpressure_tma"]["link"] == 1
