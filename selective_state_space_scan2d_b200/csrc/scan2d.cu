@@ -350,30 +350,47 @@ int launch(KernelFn fn, int threads, const Params& prm, const TmaMaps& tm, size_
 }
 
 // Can clusters of `nseg` blocks of this kernel be resident at all on this device?
-bool cluster_fits(KernelFn fn, int threads, size_t smem, int nseg) {
-  if (nseg > kMaxCluster) return false;
-  if (!allow_smem(fn, smem)) return false;
-  if (nseg > 8 && cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
-    cudaGetLastError();
-    return false;
+// How many clusters of `nseg` blocks of this kernel can be resident at once (0 if none).
+// Cached per (kernel, threads, shared memory, cluster size): the query is not free.
+int clusters_resident(KernelFn fn, int threads, size_t smem, int nseg) {
+  if (nseg > kMaxCluster) return 0;
+  static std::mutex mu;
+  static std::map<std::pair<std::pair<const void*, int>, std::pair<size_t, int>>, int> cache;
+  const auto key = std::make_pair(std::make_pair(reinterpret_cast<const void*>(fn), threads), std::make_pair(smem, nseg));
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(nseg, 1, 1);
-  cfg.blockDim = dim3(threads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = nseg;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
-    cudaGetLastError();
-    return false;
+  if (allow_smem(fn, smem) &&
+      (nseg <= 8 || cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess)) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(nseg, 1, 1);
+    cfg.blockDim = dim3(threads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = nseg;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) n = 0;
   }
-  return n > 0;
+  cudaGetLastError();
+  std::lock_guard<std::mutex> lk(mu);
+  cache[key] = n;
+  return n;
+}
+
+// Clusters are used when they fit and the last wave of clusters is not mostly empty: the
+// blocks of a chain run at the pace of its slowest block, so a partial wave costs a whole one.
+bool cluster_worth_it(KernelFn fn, int threads, size_t smem, int nseg, int chains) {
+  const int n = clusters_resident(fn, threads, smem, nseg);
+  if (n <= 0) return false;
+  const long long waves = (chains + n - 1) / n;
+  return waves == 1 || chains * 100 >= waves * n * 85;   // one wave, or >= 85% of the slots busy
 }
 
 int forward(const void* x, const void* delta, const float* A, const void* B, const void* C,
@@ -406,7 +423,8 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
   }
   // a chain's blocks share distributed shared memory when such a cluster fits on the device
   if (cp.link == kLinkCluster &&
-      !cluster_fits(tma ? cp.pl.var.fn_tma : cp.pl.var.fn_plain, cp.pl.warps * 32, cp.smem, cp.pl.nseg))
+      !cluster_worth_it(tma ? cp.pl.var.fn_tma : cp.pl.var.fn_plain, cp.pl.warps * 32, cp.smem, cp.pl.nseg,
+                        cp.pl.n_chains))
     cp = plan_call(s, tma, false);
   const Plan& pl = cp.pl;
   const KernelFn fn = tma ? pl.var.fn_tma : pl.var.fn_plain;

@@ -233,24 +233,29 @@ __device__ __noinline__ bool wait_geq(const unsigned long long* p, unsigned long
   }
 }
 
-// Bounded wait for phase `parity` of an mbarrier (TMA completion or a carry ring slot).
-// `aborted` (per warp) short-cuts every later wait once one has timed out.
-__device__ __noinline__ void mbar_wait(uint32_t bar, unsigned parity, unsigned long long* ctrl,
-                                       unsigned long long gen, long long timeout_ns, bool& aborted) {
-  if (aborted) return;
-  long long t0 = 0;
-  for (unsigned it = 0;; ++it) {
-    if (mbar_try_wait(bar, parity)) return;
+// Slow path of a bounded mbarrier wait: keeps trying until phase `parity` completes or the
+// time runs out.  Returns false after a time-out (the error is recorded).
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, unsigned parity, unsigned long long* ctrl,
+                                            unsigned long long gen, long long timeout_ns) {
+  const long long t0 = global_ns();
+  for (unsigned it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
     if ((it & 15u) == 0u) {
-      const long long now = global_ns();
-      if (it == 0u) t0 = now;
-      if (now - t0 > timeout_ns || it > (1u << 28)) {
+      if (global_ns() - t0 > timeout_ns || it > (1u << 28)) {
         report_timeout(ctrl, gen);
-        aborted = true;
-        return;
+        return false;
       }
     }
   }
+}
+
+// Bounded wait for phase `parity` of an mbarrier (TMA completion or a carry ring slot): one
+// try inline, the rest out of line.  Once a wait of this warp has timed out (`aborted`),
+// later waits return at once.  Returns the new `aborted`.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, unsigned parity, unsigned long long* ctrl,
+                                          unsigned long long gen, long long timeout_ns, bool aborted) {
+  if (aborted || mbar_try_wait(bar, parity)) return aborted;
+  return !mbar_wait_slow(bar, parity, ctrl, gen, timeout_ns);
 }
 
 // ---- staged-row element access ------------------------------------------------------------
@@ -555,8 +560,8 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
 
       // ---- (1) this row's tile is in shared memory -----------------------------------
       if (TMA) {
-        mbar_wait(smem_u32(&s_tma_bar[warp][s]), static_cast<unsigned>((u / DEPTH) & 1), p.ctrl, p.gen,
-                  p.timeout_ns, aborted);
+        aborted = mbar_wait(smem_u32(&s_tma_bar[warp][s]), static_cast<unsigned>((u / DEPTH) & 1), p.ctrl,
+                            p.gen, p.timeout_ns, aborted);
       } else {
         Tin* dst = reinterpret_cast<Tin*>(tiles);
 #pragma unroll
@@ -578,7 +583,7 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
 #pragma unroll
           for (int g = 0; g < NG; ++g) hh[c][g] = ok ? __ldcg(src + c * NG + g) : 0.f;
       } else if (has_left) {
-        mbar_wait(smem_u32(&s_full[warp][cs]), cpar, p.ctrl, p.gen, p.timeout_ns, aborted);
+        aborted = mbar_wait(smem_u32(&s_full[warp][cs]), cpar, p.ctrl, p.gen, p.timeout_ns, aborted);
         const float4* src = reinterpret_cast<const float4*>(carry_slot(warp, cs)) + lane * (L::CARRY_PAD / 4);
         float in[L::CARRY_PAD];
 #pragma unroll
@@ -668,7 +673,7 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
       if (next_local || (next_remote && cluster)) {
         // the slot is free once the consumer released its previous use
         if (u >= kCarryRing)
-          mbar_wait(my_empty0 + cs * 8, cpar ^ 1u, p.ctrl, p.gen, p.timeout_ns, aborted);
+          aborted = mbar_wait(my_empty0 + cs * 8, cpar ^ 1u, p.ctrl, p.gen, p.timeout_ns, aborted);
         float out[L::CARRY_PAD];
 #pragma unroll
         for (int e = L::CARRY; e < L::CARRY_PAD; ++e) out[e] = 0.f;
@@ -781,8 +786,8 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
     const int issued = U < u + DEPTH ? U : u + DEPTH;      // rows whose copies were started
     bool drain_gave_up = false;
     for (int uu = issued - DEPTH < 0 ? 0 : issued - DEPTH; uu < issued; ++uu)
-      mbar_wait(smem_u32(&s_tma_bar[warp][uu % DEPTH]), static_cast<unsigned>((uu / DEPTH) & 1), p.ctrl,
-                p.gen, p.timeout_ns, drain_gave_up);
+      drain_gave_up = mbar_wait(smem_u32(&s_tma_bar[warp][uu % DEPTH]), static_cast<unsigned>((uu / DEPTH) & 1),
+                                p.ctrl, p.gen, p.timeout_ns, drain_gave_up);
   }
 
   // ---- kSmemMulti: write the accumulated maps of this block's chains --------------------------
