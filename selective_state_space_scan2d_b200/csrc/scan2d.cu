@@ -423,7 +423,7 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
   }
   // a chain's blocks share distributed shared memory when such a cluster fits on the device
   if (cp.link == kLinkCluster &&
-      !cluster_worth_it(tma ? cp.pl.var.fn_tma : cp.pl.var.fn_plain, cp.pl.warps * 32, cp.smem, cp.pl.nseg,
+      !cluster_worth_it(tma ? cp.pl.var.fn_tma : cp.pl.var.fn_plain, (cp.pl.warps + (tma ? 1 : 0)) * 32, cp.smem, cp.pl.nseg,
                         cp.pl.n_chains))
     cp = plan_call(s, tma, false);
   const Plan& pl = cp.pl;
@@ -448,7 +448,7 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
       // a chain's blocks must be able to be resident together (producer back-pressure)
       int per_sm = 0;
       if (!allow_smem(fn, cp.smem)) return SCAN2D_E_LAUNCH;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, pl.warps * 32, cp.smem) != cudaSuccess) {
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, (pl.warps + (tma ? 1 : 0)) * 32, cp.smem) != cudaSuccess) {
         cudaGetLastError();
         return SCAN2D_E_LAUNCH;
       }
@@ -472,7 +472,7 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
     return ++ws->gen;
   };
 
-  const int threads = pl.warps * 32;
+  const int threads = (pl.warps + (tma ? 1 : 0)) * 32;   // + the TMA producer warp
   const int cluster = cp.link == kLinkCluster ? pl.nseg : 1;
   if (!cp.global_multi) {
     prm.mode = cp.smem_multi ? kSmemMulti : kSingle;
@@ -517,7 +517,7 @@ int scan2d_query_plan(int batch, int channels, int H, int W, int N, unsigned fla
   // global ring if such a cluster cannot be resident on the device)
   const scan2d::CallPlan cp = scan2d::plan_call(s, tma, true);
   const long long v[SCAN2D_PLAN_FIELDS] = {
-      cp.launches, cp.grid, cp.pl.warps * 32, static_cast<long long>(cp.smem), cp.pl.nseg,
+      cp.launches, cp.grid, (cp.pl.warps + (tma ? 1 : 0)) * 32, static_cast<long long>(cp.smem), cp.pl.nseg,
       cp.pl.var.cmax, cp.pl.wpc, cp.smem_multi ? 1 : (cp.global_multi ? 2 : 0), cp.pl.var.ng,
       static_cast<long long>(cp.ws_bytes), cp.pl.var.g, tma ? 1 : 0, cp.link};
   for (int k = 0; k < n_out && k < SCAN2D_PLAN_FIELDS; ++k) out[k] = v[k];

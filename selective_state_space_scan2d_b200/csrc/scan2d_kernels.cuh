@@ -53,7 +53,7 @@ constexpr int kQ = 4;                  // state-group lanes per channel group
 constexpr int kGroups = 8;             // channel groups per warp
 constexpr int kRing = 16;              // carry rows buffered in global memory between blocks
 constexpr int kCarryRing = 4;          // carry rows buffered in shared memory between warps
-constexpr int kMaxWarps = 8;           // warps per block
+constexpr int kMaxWarps = 8;           // compute warps per block (plus one TMA producer warp)
 constexpr int kDepth = 4;              // rows staged ahead per warp (TMA path)
 constexpr int kPublish = 4;            // global fallback: rows per flag release
 constexpr float kLog2e = 1.4426950408889634f;
@@ -181,6 +181,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, unsigned parity) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Non-blocking test of phase `parity` of an mbarrier.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
@@ -341,9 +354,82 @@ __host__ __device__ constexpr size_t carry_ring_bytes(int warps) {
   return static_cast<size_t>(warps) * kCarryRing * Layout<Tin, NG, G, CMAX>::CARRY_SLOT_BYTES;
 }
 
+// ---- the TMA producer warp ---------------------------------------------------------------------
+// Lane wq stages, for compute warp wq of the block, the rows of its walk into that warp's ring of
+// DEPTH tile slots: row uu goes to slot uu % DEPTH once the warp has released row uu - DEPTH.  The
+// lanes run independently, so a slow compute warp never holds up the others.  Gives up (recording
+// a time-out) when no slot of any warp frees up for timeout_ns.  issued[wq] ends as the number of
+// rows staged for warp wq.  Called by all 32 lanes of the producer warp.
+template <typename Tin, int NG, int G, int CMAX, int DEPTH>
+__device__ __noinline__ void produce_rows(const Params& p, const TmaMaps& tm, unsigned char* tiles0,
+                                          uint64_t* tfull, uint64_t* tempty, int* issued, int* abort_flag,
+                                          int ncomp, int first_strip, int chain0, int U) {
+  static_assert((DEPTH & (DEPTH - 1)) == 0, "ring depth must be a power of two");
+  using L = Layout<Tin, NG, G, CMAX>;
+  const unsigned FULL = 0xffffffffu;
+  const int wq = threadIdx.x & 31;
+  int total = 0, us = 0, bq = 0, gq = 0;
+  if (wq < ncomp) {
+    const int sl = wq / p.wpc;                         // chain slot of the warp
+    const int cq = chain0 + sl;
+    us = first_strip + (wq - sl * p.wpc);              // its strip, in scan order
+    if (cq < p.n_chains && us < p.strips) {
+      total = U;
+      bq = cq / p.n_cgroups;
+      gq = cq - bq * p.n_cgroups;
+    }
+  }
+  const uint32_t full0 = smem_u32(tfull + wq * kDepth);
+  const uint32_t empty0 = smem_u32(tempty + wq * kDepth);
+  unsigned char* ring = tiles0 + wq * DEPTH * L::TILE_BYTES;
+  int uu = 0, oi = 0, r = 0;                           // next row, as (orientation, scan row)
+  unsigned idle = 0;
+  long long t_idle = 0;
+  while (!__all_sync(FULL, uu >= total)) {
+    bool progressed = false;
+    if (uu < total) {
+      const int s = uu & (DEPTH - 1);
+      if (uu < DEPTH || mbar_test_wait(empty0 + s * 8, static_cast<unsigned>(((uu / DEPTH) - 1) & 1))) {
+        const int o = p.orient_code[oi];
+        const int i = (o & 2) ? p.H - 1 - r : r;           // stored row
+        const int t = (o & 1) ? p.strips - 1 - us : us;    // stored strip
+        const int k = p.orient_k[oi];
+        unsigned char* dst = ring + s * L::TILE_BYTES;
+        uint64_t* bar = tfull + wq * kDepth + s;
+        mbar_expect_tx(bar, L::TX_BYTES);
+        tma_load_4d(dst + L::X_OFF * L::ESZ, &tm.x, bar, t * CMAX, i, gq * L::CPW, bq);
+        tma_load_4d(dst + L::D_OFF * L::ESZ, &tm.d, bar, t * CMAX, i, gq * L::CPW, bq);
+        tma_load_4d(dst + L::B_OFF * L::ESZ, &tm.b, bar, t * CMAX, i, 0, bq * p.K + k);
+        tma_load_4d(dst + L::C_OFF * L::ESZ, &tm.c, bar, t * CMAX, i, 0, bq * p.K + k);
+        ++uu;
+        if (++r == p.H) { r = 0; ++oi; }
+        progressed = true;
+      }
+    }
+    (void)full0;
+    if (__any_sync(FULL, progressed)) {
+      idle = 0;
+    } else {
+      // nothing to stage right now: step aside for the compute warps, and give up (on every
+      // lane together) if no slot has freed up for the time limit
+      __nanosleep(32);
+      if (++idle == 1) t_idle = global_ns();
+      const bool late = (idle & 255u) == 0u && global_ns() - t_idle > p.timeout_ns;
+      if (__any_sync(FULL, late)) {
+        if (wq == 0) {
+          report_timeout(p.ctrl, p.gen);
+          *abort_flag = 1;
+        }
+        break;
+      }
+    }
+  }
+  if (wq < ncomp) issued[wq] = uu;
+}
+
 // ---- the kernel ------------------------------------------------------------------------------
 template <typename Tin, int NG, int G, int CMAX, bool TMA>
-__global__ void __launch_bounds__(kMaxWarps * 32)
+__global__ void __launch_bounds__((kMaxWarps + 1) * 32)
 scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps tm) {
   using L = Layout<Tin, NG, G, CMAX>;
   constexpr int PV = Elem<Tin>::kPerVec;
@@ -356,37 +442,41 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   constexpr int NP = L::NP;
 
   extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ uint64_t s_tma_bar[kMaxWarps][kDepth];
+  __shared__ uint64_t s_tfull[kMaxWarps][kDepth];            // staged row landed (TMA)
+  __shared__ uint64_t s_tempty[kMaxWarps][kDepth];           // staged row consumed
   __shared__ uint64_t s_full[kMaxWarps][kCarryRing];         // carry slot written (consumer side)
   __shared__ uint64_t s_empty[kMaxWarps][kCarryRing];        // carry slot read (producer side)
   __shared__ int s_item;
+  __shared__ int s_abort;
 
   const unsigned FULL = 0xffffffffu;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const int nwarps = blockDim.x >> 5;
-  const int slot = warp / p.wpc;            // chain slot inside the block
-  const int w = warp - slot * p.wpc;        // strip inside the segment
+  // compute warps 0 .. ncomp-1; with TMA one more warp issues every copy of the block
+  const int ncomp = p.wpc * p.chains_per_block;
+  const bool is_compute = warp < ncomp;
+  const int slot = is_compute ? warp / p.wpc : 0;            // chain slot inside the block
+  const int w = is_compute ? warp - slot * p.wpc : 0;        // strip inside the segment
   const int cg = lane >> 2;                 // channel group
   const int q = lane & 3;                   // state group
   const bool cluster = p.link == kLinkCluster;
   const bool global_link = p.link == kLinkGlobal;
 
   // ---- which chain and segment -------------------------------------------------------
-  int chain, seg;
-  if (cluster) {
-    seg = static_cast<int>(cluster_rank());
-    chain = blockIdx.x / p.nseg;
-  } else if (global_link) {
-    if (threadIdx.x == 0) s_item = static_cast<int>(atomicAdd(&p.ctrl[0], 1ull));
-    __syncthreads();
-    chain = s_item / p.nseg;
-    seg = s_item - chain * p.nseg;
-  } else {
-    chain = blockIdx.x * p.chains_per_block + slot;
-    seg = 0;
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    if (global_link) s_item = static_cast<int>(atomicAdd(&p.ctrl[0], 1ull));
   }
-  const bool chain_ok = chain < p.n_chains && slot < p.chains_per_block;
+  __syncthreads();
+  const int seg = cluster ? static_cast<int>(cluster_rank()) : (global_link ? s_item % p.nseg : 0);
+  // chain of chain slot `sl` of this block
+  auto chain_of = [&](int sl) -> int {
+    if (cluster) return blockIdx.x / p.nseg;
+    if (global_link) return s_item / p.nseg;
+    return blockIdx.x * p.chains_per_block + sl;
+  };
+  const int chain = chain_of(slot);
+  const bool chain_ok = is_compute && chain < p.n_chains && slot < p.chains_per_block;
   const int b = chain_ok ? chain / p.n_cgroups : 0;
   const int grp = chain_ok ? chain - b * p.n_cgroups : 0;
   const int u_scan = seg * p.wpc + w;                        // strip position in scan order
@@ -421,16 +511,19 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
 
   // ---- shared memory ---------------------------------------------------------------------
   unsigned char* carry_base = smem;
-  unsigned char* tiles = smem + carry_ring_bytes<Tin, NG, G, CMAX>(nwarps) + warp * DEPTH * L::TILE_BYTES;
-  float* yacc_s = reinterpret_cast<float*>(smem + carry_ring_bytes<Tin, NG, G, CMAX>(nwarps) +
-                                           static_cast<size_t>(nwarps) * DEPTH * L::TILE_BYTES);
+  unsigned char* tiles0 = smem + carry_ring_bytes<Tin, NG, G, CMAX>(ncomp);
+  unsigned char* tiles = tiles0 + (is_compute ? warp : 0) * DEPTH * L::TILE_BYTES;
+  float* yacc_s = reinterpret_cast<float*>(tiles0 + static_cast<size_t>(ncomp) * DEPTH * L::TILE_BYTES);
   auto carry_slot = [&](int wr, int s) -> float* {
     return reinterpret_cast<float*>(carry_base + (wr * kCarryRing + s) * L::CARRY_SLOT_BYTES);
   };
 
-  if (lane == 0) {
+  if (lane == 0 && is_compute) {
 #pragma unroll
-    for (int s = 0; s < DEPTH; ++s) mbar_init(&s_tma_bar[warp][s], 1);
+    for (int s = 0; s < DEPTH; ++s) {
+      mbar_init(&s_tfull[warp][s], 1);        // the producer's expect_tx arrival + the bytes
+      mbar_init(&s_tempty[warp][s], 32);      // every lane of the compute warp
+    }
 #pragma unroll
     for (int s = 0; s < kCarryRing; ++s) {
       mbar_init(&s_full[warp][s], 32);
@@ -442,30 +535,17 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   else __syncthreads();
 
   const int item = chain * p.nseg + seg;
-  const int U = p.orient_count * H;                          // rows this warp walks
+  const int U = p.orient_count * H;                          // rows each warp walks
 
-  // row u of the walk -> (orientation index, stored row, stored strip)
-  auto row_coords = [&](int uu, int& oi, int& i, int& t) {
+  // row uu of the walk of the warp at scan position us -> (orientation, stored row, stored strip)
+  auto row_coords_of = [&](int us, int uu, int& oi, int& i, int& t) {
     oi = uu / H;
     const int r = uu - oi * H;
     const int o = p.orient_code[oi];
     i = (o & 2) ? H - 1 - r : r;
-    t = (o & 1) ? p.strips - 1 - u_scan : u_scan;
+    t = (o & 1) ? p.strips - 1 - us : us;
   };
-
-  auto issue_tma = [&](int uu) {
-    int oi, i, t;
-    row_coords(uu, oi, i, t);
-    const int k = p.orient_k[oi];
-    const int s = uu % DEPTH;
-    unsigned char* dst = tiles + s * L::TILE_BYTES;
-    uint64_t* bar = &s_tma_bar[warp][s];
-    mbar_expect_tx(bar, L::TX_BYTES);
-    tma_load_4d(dst + L::X_OFF * L::ESZ, &tm.x, bar, t * CMAX, i, grp * L::CPW, b);
-    tma_load_4d(dst + L::D_OFF * L::ESZ, &tm.d, bar, t * CMAX, i, grp * L::CPW, b);
-    tma_load_4d(dst + L::B_OFF * L::ESZ, &tm.b, bar, t * CMAX, i, 0, b * p.K + k);
-    tma_load_4d(dst + L::C_OFF * L::ESZ, &tm.c, bar, t * CMAX, i, 0, b * p.K + k);
-  };
+  auto row_coords = [&](int uu, int& oi, int& i, int& t) { row_coords_of(u_scan, uu, oi, i, t); };
 
   // plain-load path: this lane's share of row u's tile, zero outside the tensors.  Value e
   // of the dense tile goes to tile offset plain_dst(e).
@@ -514,13 +594,15 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   };
 
   bool aborted = false;
-  if (strip_ok) {
-    if (TMA) {
-      if (lane == 0)
-        for (int uu = 0; uu < DEPTH && uu < U; ++uu) issue_tma(uu);
-    } else {
-      plain_load(0);
-    }
+  if (!TMA && strip_ok) plain_load(0);
+
+  // ---- the TMA producer warp: stages rows for every compute warp, never blocking on one ----
+  __shared__ int s_issued[kMaxWarps];                        // rows staged per compute warp
+  if (TMA && !is_compute) {
+    const int first = seg * p.wpc;
+    const int c0 = chain_of(0);
+    produce_rows<Tin, NG, G, CMAX, DEPTH>(p, tm, tiles0, &s_tfull[0][0], &s_tempty[0][0], s_issued, &s_abort,
+                                          ncomp, first, c0, U);
   }
 
   // where this warp's carries go: the next warp of this block, or warp 0 of the next block
@@ -560,7 +642,7 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
 
       // ---- (1) this row's tile is in shared memory -----------------------------------
       if (TMA) {
-        aborted = mbar_wait(smem_u32(&s_tma_bar[warp][s]), static_cast<unsigned>((u / DEPTH) & 1), p.ctrl,
+        aborted = mbar_wait(smem_u32(&s_tfull[warp][s]), static_cast<unsigned>((u / DEPTH) & 1), p.ctrl,
                             p.gen, p.timeout_ns, aborted);
       } else {
         Tin* dst = reinterpret_cast<Tin*>(tiles);
@@ -662,12 +744,9 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
         for (int vg = NVEC - 1; vg >= 0; --vg) vec_group(vg, true);
       }
 
-      // ---- (4) the tile slot is free again: stage row u + DEPTH into it ---------------------
-      __syncwarp();
-      if (TMA && lane == 0 && u + DEPTH < U) {
-        fence_proxy_async();
-        issue_tma(u + DEPTH);
-      }
+      // ---- (4) the tile slot is free again: tell the producer warp (every lane has read) ------
+      if (TMA) mbar_arrive_local(smem_u32(&s_tempty[warp][s]));
+      else __syncwarp();
 
       // ---- (5) carry-out to the next strip ---------------------------------------------------
       if (next_local || (next_remote && cluster)) {
@@ -776,18 +855,21 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
         }
       }
     }
-    // orientations summed in shared memory: no warp may start the next orientation (whose
-    // strips map to other columns) before every warp has finished this one
-    if (p.mode == kSmemMulti) __syncthreads();
+    // orientations summed in shared memory: no compute warp may start the next orientation
+    // (whose strips map to other columns) before every compute warp has finished this one
+    if (p.mode == kSmemMulti && is_compute)
+      asm volatile("bar.sync 1, %0;" ::"r"(ncomp * 32) : "memory");
   }
+  if (aborted) s_abort = 1;
+  __syncthreads();
 
-  // ---- after a timed-out wait: let this warp's TMA copies still in flight land (bounded) ------
-  if (TMA && aborted && strip_ok && lane == 0) {
-    const int issued = U < u + DEPTH ? U : u + DEPTH;      // rows whose copies were started
-    bool drain_gave_up = false;
-    for (int uu = issued - DEPTH < 0 ? 0 : issued - DEPTH; uu < issued; ++uu)
-      drain_gave_up = mbar_wait(smem_u32(&s_tma_bar[warp][uu % DEPTH]), static_cast<unsigned>((uu / DEPTH) & 1),
-                                p.ctrl, p.gen, p.timeout_ns, drain_gave_up);
+  // ---- after a timed-out wait: let the copies still in flight land (bounded) ------------------
+  if (TMA && !is_compute && lane == 0 && s_abort) {
+    bool gave_up = false;
+    for (int wq = 0; wq < ncomp; ++wq)
+      for (int uu = s_issued[wq] - DEPTH < 0 ? 0 : s_issued[wq] - DEPTH; uu < s_issued[wq]; ++uu)
+        gave_up = mbar_wait(smem_u32(&s_tfull[wq][uu % DEPTH]), static_cast<unsigned>((uu / DEPTH) & 1),
+                            p.ctrl, p.gen, p.timeout_ns, gave_up);
   }
 
   // ---- kSmemMulti: write the accumulated maps of this block's chains --------------------------
