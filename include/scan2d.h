@@ -66,6 +66,7 @@ extern "C" {
 
 /* ---- limits ---------------------------------------------------------------------- */
 #define SCAN2D_MAX_N    64     /* states per channel                                   */
+#define SCAN2D_NOALLOC_SCRATCH_BYTES 33554432  /* fixed scratch of scan2d_fwd_noalloc (32 MiB) */
 
 /* ---- error codes ----------------------------------------------------------------- */
 #define SCAN2D_OK          0
@@ -79,6 +80,8 @@ extern "C" {
 #define SCAN2D_E_NOMEM    -8   /* the internal workspace could not be allocated         */
 #define SCAN2D_E_DEVICE   -9   /* no usable CUDA device, or not an sm_100 device        */
 #define SCAN2D_E_STAGING -10   /* scan2d_fwd_host: staging buffer too small             */
+#define SCAN2D_E_SCRATCH -11   /* scan2d_fwd_noalloc: shape needs more scratch than the
+                                  fixed SCAN2D_NOALLOC_SCRATCH_BYTES                    */
 
 /*
  * scan2d_fwd -- the 2D selective-scan forward on device buffers.
@@ -93,6 +96,34 @@ extern "C" {
 int scan2d_fwd(const void *x, const void *delta, const float *A, const void *B, const void *C,
                const float *Dskip, void *y, int batch, int channels, int H, int W, int N,
                unsigned flags, void *stream);
+
+/*
+ * scan2d_fwd_noalloc -- scan2d_fwd for callers that must not allocate device memory.  The
+ * pages have no counterpart: this entry point exists for the host program, not the method.
+ * Some callers cannot let a library call cudaMalloc: a runtime whose allocator has already
+ * reserved the device memory it may use (a cudaMalloc outside it can fail or fragment it),
+ * a plugin or operator interface that forbids allocating inside its execute call, or a
+ * latency-bound loop that cannot afford the device-wide synchronisation cudaMalloc and
+ * cudaFree may cause.  scan2d_fwd keeps a per-stream workspace that it allocates on first
+ * need; this entry point instead takes its scratch (cross-block carry rings, and the fp32
+ * accumulator of several orientations with bf16 output on maps too large for shared memory)
+ * from one fixed device array of SCAN2D_NOALLOC_SCRATCH_BYTES that the library holds on every
+ * device that loads it, until the process exits.  It calls no cudaMalloc, cudaFree or other
+ * allocating routine.  Arguments, layouts and results are those of scan2d_fwd (y is
+ * bitwise the same for the same launch plan).
+ *   - The first call on a device looks up the array's device address with that device
+ *     current; make that first call before any stream capture.
+ *   - Every call, on every stream, shares the one array and leaves its contents behind; each
+ *     call clears (cudaMemsetAsync on `stream`) the words that must start at zero.  Calls
+ *     whose work overlaps on the GPU (different streams, or other threads) race on the
+ *     array and give undefined results: order them, e.g. on one stream.
+ *   - A shape whose scratch exceeds SCAN2D_NOALLOC_SCRATCH_BYTES (see scan2d_query_plan
+ *     field [9]) is rejected with SCAN2D_E_SCRATCH before anything is enqueued.
+ * Returns the scan2d_fwd codes (never SCAN2D_E_NOMEM), or SCAN2D_E_SCRATCH.
+ */
+int scan2d_fwd_noalloc(const void *x, const void *delta, const float *A, const void *B,
+                       const void *C, const float *Dskip, void *y, int batch, int channels,
+                       int H, int W, int N, unsigned flags, void *stream);
 
 /*
  * scan2d_query_plan -- how scan2d_fwd would run a call of this shape, without launching

@@ -393,9 +393,11 @@ bool cluster_worth_it(KernelFn fn, int threads, size_t smem, int nseg, int chain
   return waves == 1 || chains * 100 >= waves * n * 85;   // one wave, or >= 85% of the slots busy
 }
 
+// `fixed_scratch`, when given, is the device address of a buffer of
+// SCAN2D_NOALLOC_SCRATCH_BYTES that replaces the per-stream workspace (nothing is allocated).
 int forward(const void* x, const void* delta, const float* A, const void* B, const void* C,
             const float* Dskip, void* y, int batch, int channels, int H, int W, int N,
-            unsigned flags, cudaStream_t st) {
+            unsigned flags, cudaStream_t st, char* fixed_scratch = nullptr) {
   Shape s;
   int rc = check_shape(batch, channels, H, W, N, flags, &s);
   if (rc) return rc;
@@ -454,10 +456,24 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
       }
       if (static_cast<long long>(per_sm) * nsm < pl.nseg) return SCAN2D_E_DIMS;
     }
-    ws = get_workspace(dev, st, cp.link == kLinkGlobal ? cp.items : 0, cp.carry_bytes + cp.yacc_bytes);
-    if (!ws) return SCAN2D_E_NOMEM;
-    char* base = static_cast<char*>(ws->ptr);
-    const size_t cap = ws->cap_items;
+    char* base = nullptr;
+    size_t cap = 0;
+    if (fixed_scratch != nullptr) {
+      // the fixed buffer keeps the previous call's contents: its control, flag and ack
+      // words are cleared for every call, which then starts again at generation 1
+      if (cp.ws_bytes > SCAN2D_NOALLOC_SCRATCH_BYTES) return SCAN2D_E_SCRATCH;
+      base = fixed_scratch;
+      cap = cp.link == kLinkGlobal ? cp.items : 0;
+      if (cudaMemsetAsync(base, 0, sync_bytes(cap), st) != cudaSuccess) {
+        cudaGetLastError();
+        return SCAN2D_E_LAUNCH;
+      }
+    } else {
+      ws = get_workspace(dev, st, cp.link == kLinkGlobal ? cp.items : 0, cp.carry_bytes + cp.yacc_bytes);
+      if (!ws) return SCAN2D_E_NOMEM;
+      base = static_cast<char*>(ws->ptr);
+      cap = ws->cap_items;
+    }
     prm.ctrl = reinterpret_cast<unsigned long long*>(base);
     prm.flags = reinterpret_cast<unsigned long long*>(base + kAlign);
     prm.acks = reinterpret_cast<unsigned long long*>(base + kAlign + round_up(cap * 8, kAlign));
@@ -493,6 +509,31 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
   return SCAN2D_OK;
 }
 
+// ---- fixed scratch for callers that cannot allocate device memory -------------------------
+// One buffer per device, allocated by the CUDA runtime when the library's module is loaded
+// and held until the process exits.  Host code must not use the array's name as a device
+// address: the address is looked up once per device with that device current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SCAN2D_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+char* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device `dev`, or null.
+char* noalloc_scratch(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_noalloc_addr[dev] = static_cast<char*>(p);
+  }
+  return g_noalloc_addr[dev];
+}
+
 }  // namespace scan2d
 
 // ---- C ABI ---------------------------------------------------------------------------------
@@ -503,6 +544,22 @@ int scan2d_fwd(const void* x, const void* delta, const float* A, const void* B, 
                unsigned flags, void* stream) {
   return scan2d::forward(x, delta, A, B, C, Dskip, y, batch, channels, H, W, N, flags,
                          static_cast<cudaStream_t>(stream));
+}
+
+int scan2d_fwd_noalloc(const void* x, const void* delta, const float* A, const void* B,
+                       const void* C, const float* Dskip, void* y, int batch, int channels, int H,
+                       int W, int N, unsigned flags, void* stream) {
+  scan2d::Shape s;
+  int rc = scan2d::check_shape(batch, channels, H, W, N, flags, &s);
+  if (rc) return rc;
+  if (!x || !delta || !A || !B || !C || !y) return SCAN2D_E_NULL;
+  int dev = 0, nsm = 0;
+  rc = scan2d::device_ok(&dev, &nsm);
+  if (rc) return rc;
+  char* scratch = scan2d::noalloc_scratch(dev);
+  if (scratch == nullptr) return SCAN2D_E_DEVICE;
+  return scan2d::forward(x, delta, A, B, C, Dskip, y, batch, channels, H, W, N, flags,
+                         static_cast<cudaStream_t>(stream), scratch);
 }
 
 int scan2d_query_plan(int batch, int channels, int H, int W, int N, unsigned flags,
@@ -610,6 +667,7 @@ const char* scan2d_strerror(int code) {
     case SCAN2D_E_NOMEM: return "workspace allocation failed";
     case SCAN2D_E_DEVICE: return "no usable sm_100 CUDA device";
     case SCAN2D_E_STAGING: return "staging buffer too small";
+    case SCAN2D_E_SCRATCH: return "scan2d_fwd_noalloc: the shape needs more scratch than SCAN2D_NOALLOC_SCRATCH_BYTES";
     default: return "unknown error";
   }
 }

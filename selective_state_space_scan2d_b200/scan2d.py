@@ -27,6 +27,8 @@ _lib = ctypes.CDLL(lib_path)
 _vp, _i, _u, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_size_t
 _lib.scan2d_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _u, _vp]
 _lib.scan2d_fwd.restype = _i
+_lib.scan2d_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _u, _vp]
+_lib.scan2d_fwd_noalloc.restype = _i
 _lib.scan2d_query_plan.argtypes = [_i, _i, _i, _i, _i, _u, ctypes.POINTER(ctypes.c_longlong), _i]
 _lib.scan2d_query_plan.restype = _i
 _lib.scan2d_host_staging_bytes.argtypes = [_i, _i, _i, _i, _i, _u]
@@ -47,6 +49,8 @@ SCAN2D_OR_TL = 0x10
 SCAN2D_OR_TR = 0x20
 SCAN2D_OR_BL = 0x40
 SCAN2D_OR_BR = 0x80
+SCAN2D_E_SCRATCH = -11
+SCAN2D_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class Scan2dError(RuntimeError):
@@ -140,6 +144,28 @@ def scan2d_fwd(x, delta, A, B, C, Dskip=None, y=None, flags=None, stream=None):
                          batch, D, H, W, N, flags, _stream_handle(stream))
     if rc:
         raise Scan2dError(rc, "scan2d_fwd")
+    return y
+
+
+def scan2d_fwd_noalloc(x, delta, A, B, C, Dskip, y, flags=None, stream=None):
+    """scan2d_fwd into a caller-provided y, with the library's fixed device scratch instead of
+    an allocated workspace: for callers that must not allocate device memory (a runtime whose
+    allocator owns the device's memory, an operator interface that forbids allocating during
+    execution, a loop that cannot take the synchronisation an allocation may cause).  Calls
+    share that scratch, so calls that overlap on the GPU race; shapes that need more than
+    SCAN2D_NOALLOC_SCRATCH_BYTES raise Scan2dError (SCAN2D_E_SCRATCH)."""
+    torch = _torch()
+    _check(x, delta, A, B, C, Dskip, "cuda")
+    batch, D, H, W, N, K = _dims(x, B, A)
+    if flags is None:
+        flags = flags_for(x.dtype == torch.bfloat16, (1 << K) - 1)
+    out_dtype = torch.float32 if (x.dtype == torch.float32 or flags & SCAN2D_OUT_F32) else torch.bfloat16
+    if y is None or y.dtype != out_dtype or tuple(y.shape) != (batch, D, H, W) or not y.is_contiguous():
+        raise ValueError("y must be a contiguous CUDA tensor of the output dtype and shape")
+    rc = _lib.scan2d_fwd_noalloc(_ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(Dskip),
+                                 _ptr(y), batch, D, H, W, N, flags, _stream_handle(stream))
+    if rc:
+        raise Scan2dError(rc, "scan2d_fwd_noalloc")
     return y
 
 
