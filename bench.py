@@ -66,6 +66,46 @@ def roofline_model(w: inputs.Workload):
                 roof_gelem=1e-9 / max(t_hbm, t_sfu, t_fp32))
 
 
+METRIC = "2D selective-scan fwd Gelem/s (B*D*H*W) and % of HBM/SFU roofline"
+
+
+def base_config(w: inputs.Workload, world: int) -> dict:
+    return {"workload": w.name, "batch": w.batch, "channels": w.channels, "N": w.N,
+            "H": w.H, "W": w.W, "dtype_in": w.dtype, "orientations": w.K,
+            "global_batch": w.batch * world, "parallelism": f"replicas x{world}"}
+
+
+KERNEL_SOURCES = ("selective_state_space_scan2d_b200/csrc/scan2d.cu",
+                  "selective_state_space_scan2d_b200/csrc/scan2d_kernels.cuh")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "scan2d_dram_traffic.txt")
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def dram_traffic(w: inputs.Workload):
+    """DRAM bytes (read + write) per launch of the scan kernel for this workload, from the
+    committed ncu summary; None when there is none or the kernel sources changed since."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            lines = [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
+    except OSError:
+        return None
+    key = f"{w.name}:{w.batch}x{w.channels}x{w.H}x{w.W}"
+    src = kernel_source_hash()
+    for parts in lines:
+        # <workload:BxDxHxW> <kernel source hash> <bytes per launch> ...
+        if len(parts) >= 3 and parts[0] == key and parts[1] == src:
+            return float(parts[2])
+    return None
+
+
 class ClockSampler:
     """Polls SM clock and clock-event reasons through NVML while running."""
 
@@ -184,12 +224,11 @@ def run_reference(args, w: inputs.Workload):
     value = elems / dt / 1e9
     sample = f"{per_step} whole (b,d) maps of {w.name} per step ({elems} elements), fp64 C oracle"
     print(json.dumps({
-        "impl": "reference", "metric": "2D selective-scan fwd Gelem/s (B*D*H*W)", "value": value,
+        "impl": "reference", "metric": METRIC, "value": value,
         "unit": "Gelem/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "batch": w.batch, "channels": w.channels, "N": w.N,
-                   "H": w.H, "W": w.W, "dtype_in": w.dtype, "orientations": w.K},
+        "config": base_config(w, 1),
         "cpu_baseline": {"value": value, "unit": "Gelem/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "Gelem/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
@@ -274,10 +313,21 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--others", action="store_true", help="also time the other workloads (extra key)")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--override", action="append", default=[], metavar="KEY=INT",
+                    help="change batch/channels/H/W of the workload (smaller cases for ncu captures)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer (e2e) leg")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     w = inputs.WORKLOADS[args.workload]
+    if args.override:
+        kw = {}
+        for item in args.override:
+            key, _, val = item.partition("=")
+            if key not in ("batch", "channels", "H", "W"):
+                ap.error(f"--override: unknown key {key!r}")
+            kw[key] = int(val)
+        w = w.scaled(**kw)
 
     if args.impl == "reference":
         run_reference(args, w)
@@ -299,9 +349,9 @@ def main():
                                              device_id=device)
 
     res = measure_workload(w, args, torch, scan2d, device, rank, seed=rank, steps=args.steps,
-                           warmup=args.warmup, with_e2e=True)
+                           warmup=args.warmup, with_e2e=not args.no_e2e)
     ms = res["ms"]
-    e2e_ms = res["e2e"]["ms"]
+    e2e_ms = res["e2e"]["ms"] if "e2e" in res else float("nan")
     if world > 1:
         t = torch.tensor([ms, e2e_ms], device=device, dtype=torch.float64)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
@@ -324,7 +374,7 @@ def main():
         unit = "GB/s"
     roof = {"bound": "alu" if rm["bound"] != "hbm" else "hbm", "unit_of_bound": rm["bound"],
             "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
-            "traffic": None, "peak_kind": f"nominal {SMS} SMs x {MUFU_PER_CLK_SM if rm['bound']=='sfu' else FP32_PER_CLK_SM}/clk x {rm['sm_mhz']:.0f} MHz (max clock)" if rm["bound"] != "hbm" else f"{rm['hbm_kind']} copy bandwidth",
+            "traffic": dram_traffic(w), "peak_kind": f"nominal {SMS} SMs x {MUFU_PER_CLK_SM if rm['bound']=='sfu' else FP32_PER_CLK_SM}/clk x {rm['sm_mhz']:.0f} MHz (max clock)" if rm["bound"] != "hbm" else f"{rm['hbm_kind']} copy bandwidth",
             "hbm_achieved_gbs": w.elements * rm["bytes_el"] / (ms * 1e-3) / 1e9,
             "hbm_frac_of_measured": w.elements * rm["bytes_el"] / (ms * 1e-3) / 1e9 / rm["hbm_gbs"],
             "roofline_gelem_s": rm["roof_gelem"], "frac_of_roofline_gelem": (w.elements / (ms * 1e-3) / 1e9) / rm["roof_gelem"]}
@@ -333,23 +383,23 @@ def main():
         roof["frac_at_sampled_clock"] = roof["frac"] * (rm["sm_mhz"] / clocks["sm_mhz"]) if rm["bound"] != "hbm" else roof["frac"]
 
     line = {
-        "metric": "2D selective-scan fwd Gelem/s (B*D*H*W) and % of HBM/SFU roofline",
+        "metric": METRIC,
         "value": value, "unit": "Gelem/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32" if w.dtype == "f32" else "bf16-in/f32-acc",
         "data": "synthetic",
-        "config": {"workload": w.name, "batch": w.batch, "channels": w.channels, "N": w.N,
-                   "H": w.H, "W": w.W, "dtype_in": w.dtype, "orientations": w.K,
-                   "global_batch": w.batch * world, "parallelism": f"replicas x{world}",
-                   "l2": f"inputs rotated over {res['n_sets']} device copies (> 3x L2 per rotation)"},
+        "config": {**base_config(w, world),
+                   "l2": f"inputs rotated over {res['n_sets']} device copies (> 3x L2 per rotation)",
+                   **({"overrides": args.override} if args.override else {})},
         "roofline": roof,
         "clocks": clocks,
         "gpu_launches": args.steps * res["plan"]["launches"],
         "plan": res["plan"],
-        "e2e": {"value": e2e_value, "unit": "Gelem/s", "h2d_bytes_per_step": res["e2e"]["h2d"],
-                "d2h_bytes_per_step": res["e2e"]["d2h"], "steps": res["e2e"]["steps"],
-                "api": "scan2d_fwd_host (pinned host buffers)"},
     }
+    if "e2e" in res:
+        line["e2e"] = {"value": e2e_value, "unit": "Gelem/s", "h2d_bytes_per_step": res["e2e"]["h2d"],
+                       "d2h_bytes_per_step": res["e2e"]["d2h"], "steps": res["e2e"]["steps"],
+                       "api": "scan2d_fwd_host (pinned host buffers)"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, nmaps, secs = _oracle_sample_rate(w, res["d"], args.cpu_budget)
         line["cpu_baseline"] = {"value": rate, "unit": "Gelem/s", "cores": 1, "kind": "oracle",

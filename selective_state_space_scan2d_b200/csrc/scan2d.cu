@@ -186,37 +186,40 @@ bool tma_possible(const Shape& s, const void* x, const void* delta, const void* 
 }
 
 // ---- per-(device, stream) workspace --------------------------------------------------------
-// Layout: [control words: 256 B][flags: cap_items u64][acks: cap_items u64][carry ring ...]
-// [fp32 accumulator ...].  The flag and ack words keep their place for the life of the
-// allocation (only generation-tagged values are ever written there), so a later call of
-// another shape can never read an earlier call's carry values as flags.  The region is
-// reallocated, zeroed, when a call needs more items than it holds.
+// Layout: [control words: 256 B][acks: cap_items u64][carry ring: carry_cap bytes of tagged
+// words][fp32 accumulator ...].  The ack and carry regions keep their place and size for the
+// life of the allocation and only ever hold generation-tagged words, so a later call of
+// another shape can never take an earlier call's data for its own.  The workspace is
+// reallocated, zeroed, when a call needs more than it holds, and its tagged regions are
+// zeroed again before the 20 generation bits of the carry tags wrap.
 struct Workspace {
   void* ptr = nullptr;
   size_t bytes = 0;
   size_t cap_items = 0;
+  size_t carry_cap = 0;
   unsigned long long gen = 0;
 };
 
 std::mutex g_mu;
 std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
 
-size_t sync_bytes(size_t items) { return kAlign + round_up(items * 8, kAlign) * 2; }
+size_t sync_bytes(size_t items) { return kAlign + round_up(items * 8, kAlign); }
 
-// A workspace whose flag region holds `items` items and whose tail after it holds `tail`
-// bytes, zero-initialised when (re)created, or null.
-Workspace* get_workspace(int dev, cudaStream_t st, size_t items, size_t tail) {
+// A workspace whose ack region holds `items` items, whose carry region holds `carry` bytes
+// and whose tail after them holds `tail` bytes, zero-initialised when (re)created, or null.
+Workspace* get_workspace(int dev, cudaStream_t st, size_t items, size_t carry, size_t tail) {
   std::lock_guard<std::mutex> lk(g_mu);
   Workspace& ws = g_ws[std::make_pair(dev, st)];
-  if (ws.cap_items < items || ws.bytes < sync_bytes(ws.cap_items) + tail) {
-    size_t cap = ws.cap_items;
+  if (ws.cap_items < items || ws.carry_cap < carry || ws.bytes < sync_bytes(ws.cap_items) + ws.carry_cap + tail) {
+    size_t cap = ws.cap_items, ccap = ws.carry_cap;
     if (cap < items) cap = items > 2 * cap ? items : 2 * cap;
+    if (ccap < carry) ccap = carry > 2 * ccap ? carry : 2 * ccap;
     if (ws.ptr != nullptr) {
       if (cudaStreamSynchronize(st) != cudaSuccess) return nullptr;
       cudaFree(ws.ptr);
       ws = Workspace{};
     }
-    const size_t want = round_up(sync_bytes(cap) + tail, 1 << 20);
+    const size_t want = round_up(sync_bytes(cap) + ccap + tail, 1 << 20);
     if (cudaMalloc(&ws.ptr, want) != cudaSuccess) {
       cudaGetLastError();
       ws = Workspace{};
@@ -229,6 +232,7 @@ Workspace* get_workspace(int dev, cudaStream_t st, size_t items, size_t tail) {
     }
     ws.bytes = want;
     ws.cap_items = cap;
+    ws.carry_cap = ccap;
     ws.gen = 0;
   }
   return &ws;
@@ -299,8 +303,8 @@ CallPlan plan_call(const Shape& s, bool tma, bool cluster_ok) {
   cp.global_multi = s.K > 1 && !cp.smem_multi;
   cp.need_yacc_ws = cp.global_multi && !s.out_f32;
   cp.items = static_cast<size_t>(pl.n_chains) * pl.nseg;
-  cp.carry_bytes = cp.link == kLinkGlobal
-                       ? round_up(cp.items * kRing * 32 * pl.var.g * pl.var.ng * sizeof(float), kAlign) : 0;
+  const size_t carry2 = (static_cast<size_t>(pl.var.g) * pl.var.ng + 1) / 2 * 2;   // tagged words per lane
+  cp.carry_bytes = cp.link == kLinkGlobal ? round_up(cp.items * kRing * 32 * carry2 * 8, kAlign) : 0;
   cp.yacc_bytes = cp.need_yacc_ws ? s.xy_count * sizeof(float) : 0;
   cp.need_ws = cp.link == kLinkGlobal || cp.need_yacc_ws;
   cp.ws_bytes = cp.need_ws ? sync_bytes(cp.link == kLinkGlobal ? cp.items : 0) + cp.carry_bytes + cp.yacc_bytes : 0;
@@ -425,7 +429,7 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
   }
   // a chain's blocks share distributed shared memory when such a cluster fits on the device
   if (cp.link == kLinkCluster &&
-      !cluster_worth_it(tma ? cp.pl.var.fn_tma : cp.pl.var.fn_plain, (cp.pl.warps + (tma ? 1 : 0)) * 32, cp.smem, cp.pl.nseg,
+      !cluster_worth_it(tma ? cp.pl.var.fn_tma : cp.pl.var.fn_plain, cp.pl.warps * 32, cp.smem, cp.pl.nseg,
                         cp.pl.n_chains))
     cp = plan_call(s, tma, false);
   const Plan& pl = cp.pl;
@@ -450,45 +454,52 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
       // a chain's blocks must be able to be resident together (producer back-pressure)
       int per_sm = 0;
       if (!allow_smem(fn, cp.smem)) return SCAN2D_E_LAUNCH;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, (pl.warps + (tma ? 1 : 0)) * 32, cp.smem) != cudaSuccess) {
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, pl.warps * 32, cp.smem) != cudaSuccess) {
         cudaGetLastError();
         return SCAN2D_E_LAUNCH;
       }
       if (static_cast<long long>(per_sm) * nsm < pl.nseg) return SCAN2D_E_DIMS;
     }
     char* base = nullptr;
-    size_t cap = 0;
+    size_t cap = 0, ccap = 0;
     if (fixed_scratch != nullptr) {
-      // the fixed buffer keeps the previous call's contents: its control, flag and ack
+      // the fixed buffer keeps the previous call's contents: its control, ack and carry
       // words are cleared for every call, which then starts again at generation 1
       if (cp.ws_bytes > SCAN2D_NOALLOC_SCRATCH_BYTES) return SCAN2D_E_SCRATCH;
       base = fixed_scratch;
       cap = cp.link == kLinkGlobal ? cp.items : 0;
-      if (cudaMemsetAsync(base, 0, sync_bytes(cap), st) != cudaSuccess) {
+      ccap = cp.carry_bytes;
+      if (cudaMemsetAsync(base, 0, sync_bytes(cap) + ccap, st) != cudaSuccess) {
         cudaGetLastError();
         return SCAN2D_E_LAUNCH;
       }
     } else {
-      ws = get_workspace(dev, st, cp.link == kLinkGlobal ? cp.items : 0, cp.carry_bytes + cp.yacc_bytes);
+      ws = get_workspace(dev, st, cp.link == kLinkGlobal ? cp.items : 0, cp.carry_bytes, cp.yacc_bytes);
       if (!ws) return SCAN2D_E_NOMEM;
       base = static_cast<char*>(ws->ptr);
       cap = ws->cap_items;
+      ccap = ws->carry_cap;
     }
     prm.ctrl = reinterpret_cast<unsigned long long*>(base);
-    prm.flags = reinterpret_cast<unsigned long long*>(base + kAlign);
-    prm.acks = reinterpret_cast<unsigned long long*>(base + kAlign + round_up(cap * 8, kAlign));
-    prm.carry = reinterpret_cast<float*>(base + sync_bytes(cap));
-    if (cp.need_yacc_ws) prm.yacc = reinterpret_cast<float*>(base + sync_bytes(cap) + cp.carry_bytes);
+    prm.acks = reinterpret_cast<unsigned long long*>(base + kAlign);
+    prm.carry = reinterpret_cast<unsigned long long*>(base + sync_bytes(cap));
+    if (cp.need_yacc_ws) prm.yacc = reinterpret_cast<float*>(base + sync_bytes(cap) + ccap);
   }
   if (cp.global_multi && s.out_f32) prm.yacc = static_cast<float*>(y);
 
+  // generation of the next launch; before the carry tags' 20 generation bits wrap, the
+  // tagged regions are zeroed (in stream order) and generation ...00000 is skipped
   auto next_gen = [&]() -> unsigned long long {
     if (!ws) return 1ull;
     std::lock_guard<std::mutex> lk(g_mu);
-    return ++ws->gen;
+    if (((++ws->gen) & 0xFFFFFull) == 0ull) {
+      cudaMemsetAsync(static_cast<char*>(ws->ptr) + kAlign, 0, sync_bytes(ws->cap_items) - kAlign + ws->carry_cap, st);
+      ++ws->gen;
+    }
+    return ws->gen;
   };
 
-  const int threads = (pl.warps + (tma ? 1 : 0)) * 32;   // + the TMA producer warp
+  const int threads = pl.warps * 32;
   const int cluster = cp.link == kLinkCluster ? pl.nseg : 1;
   if (!cp.global_multi) {
     prm.mode = cp.smem_multi ? kSmemMulti : kSingle;
@@ -574,7 +585,7 @@ int scan2d_query_plan(int batch, int channels, int H, int W, int N, unsigned fla
   // global ring if such a cluster cannot be resident on the device)
   const scan2d::CallPlan cp = scan2d::plan_call(s, tma, true);
   const long long v[SCAN2D_PLAN_FIELDS] = {
-      cp.launches, cp.grid, (cp.pl.warps + (tma ? 1 : 0)) * 32, static_cast<long long>(cp.smem), cp.pl.nseg,
+      cp.launches, cp.grid, cp.pl.warps * 32, static_cast<long long>(cp.smem), cp.pl.nseg,
       cp.pl.var.cmax, cp.pl.wpc, cp.smem_multi ? 1 : (cp.global_multi ? 2 : 0), cp.pl.var.ng,
       static_cast<long long>(cp.ws_bytes), cp.pl.var.g, tma ? 1 : 0, cp.link};
   for (int k = 0; k < n_out && k < SCAN2D_PLAN_FIELDS; ++k) out[k] = v[k];

@@ -97,10 +97,9 @@ struct Params {
   int vec_store;            // rows of y are aligned for 4-column vector stores
   int out_f32;              // y is fp32 (else bf16)
   unsigned long long* ctrl;   // [0] ticket counter, [1] finished blocks, [2] aborted generation
-  unsigned long long* flags;  // [n_chains*nseg] rows published by a segment (tagged)
   unsigned long long* acks;   // [n_chains*nseg] rows consumed by a segment (tagged)
-  float* carry;               // [n_chains*nseg][kRing][32][G*NG]
-  unsigned long long gen;     // launch generation, tags flags and acks
+  unsigned long long* carry;  // [n_chains*nseg][kRing][32][CARRY2] tagged carry words
+  unsigned long long gen;     // launch generation, tags acks and carry words
   long long timeout_ns;
 };
 
@@ -139,6 +138,28 @@ __device__ __forceinline__ unsigned long long tag(unsigned long long gen, int v)
   return (gen << 32) | static_cast<unsigned>(v);
 }
 
+// Global carry ring: every word is (tag << 32) | float bits, written and read as single
+// 8-byte accesses, so a word is valid exactly when its tag is the one expected and no flag
+// (with the fence it would need) guards the ring.  The tag is the low 20 bits of the launch
+// generation and the low 12 bits of row + 1; the host zeroes the ring before the
+// generation's low 20 bits wrap, and a slot is only ever refilled kRing rows later.
+__device__ __forceinline__ unsigned ctag(unsigned long long gen, int r) {
+  return (static_cast<unsigned>(gen & 0xFFFFFull) << 12) | (static_cast<unsigned>(r + 1) & 0xFFFu);
+}
+
+__device__ __forceinline__ void st_relaxed(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_relaxed_v2(unsigned long long* p, unsigned long long a, unsigned long long b) {
+  asm volatile("st.relaxed.gpu.global.v2.u64 [%0], {%1, %2};" ::"l"(p), "l"(a), "l"(b) : "memory");
+}
+
+__device__ __forceinline__ void ld_relaxed_v2(const unsigned long long* p, unsigned long long& a,
+                                              unsigned long long& b) {
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -172,8 +193,24 @@ __device__ __forceinline__ void mbar_arrive_local(uint32_t bar) {
   asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+// Relaxed arrive on another block's mbarrier: orders nothing, so it never waits for this
+// thread's outstanding global stores.  Used to free a carry slot once its values are in use.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+
+// Arms this block's mbarrier for `bytes` of st.async data (arrive + expect_tx, relaxed).
+__device__ __forceinline__ void mbar_arm_tx(uint32_t bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.relaxed.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// 16 bytes into another block's shared memory; their arrival completes `bytes` of the
+// transaction count of that block's mbarrier `cluster_bar` (no arrive, no fence).
+__device__ __forceinline__ void st_async_v4(uint32_t addr, float a, float b, float c, float d, uint32_t cluster_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+               ::"r"(addr), "r"(__float_as_uint(a)), "r"(__float_as_uint(b)), "r"(__float_as_uint(c)),
+               "r"(__float_as_uint(d)), "r"(cluster_bar)
+               : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, unsigned parity) {
@@ -199,11 +236,6 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, unsigned parity) {
       : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
-}
-
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
 }
 
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar,
@@ -340,6 +372,7 @@ struct Layout {
   static constexpr int PLAIN_PER_LANE = DENSE / 32;          // plain-load path: values per lane
   static constexpr int CARRY = G * NG;                       // carry floats per lane
   static constexpr int CARRY_PAD = (CARRY + 3) / 4 * 4;      // ... padded to whole float4s
+  static constexpr int CARRY2 = (CARRY + 1) / 2 * 2;         // tagged words per lane (global ring)
   static constexpr int CARRY_SLOT_BYTES = 32 * CARRY_PAD * 4;  // one carry row of a warp
   static constexpr int E = CMAX * G;                         // partial outputs per lane per row
   static constexpr int NP = CMAX / 2;                        // column pairs per strip
@@ -354,82 +387,9 @@ __host__ __device__ constexpr size_t carry_ring_bytes(int warps) {
   return static_cast<size_t>(warps) * kCarryRing * Layout<Tin, NG, G, CMAX>::CARRY_SLOT_BYTES;
 }
 
-// ---- the TMA producer warp ---------------------------------------------------------------------
-// Lane wq stages, for compute warp wq of the block, the rows of its walk into that warp's ring of
-// DEPTH tile slots: row uu goes to slot uu % DEPTH once the warp has released row uu - DEPTH.  The
-// lanes run independently, so a slow compute warp never holds up the others.  Gives up (recording
-// a time-out) when no slot of any warp frees up for timeout_ns.  issued[wq] ends as the number of
-// rows staged for warp wq.  Called by all 32 lanes of the producer warp.
-template <typename Tin, int NG, int G, int CMAX, int DEPTH>
-__device__ __noinline__ void produce_rows(const Params& p, const TmaMaps& tm, unsigned char* tiles0,
-                                          uint64_t* tfull, uint64_t* tempty, int* issued, int* abort_flag,
-                                          int ncomp, int first_strip, int chain0, int U) {
-  static_assert((DEPTH & (DEPTH - 1)) == 0, "ring depth must be a power of two");
-  using L = Layout<Tin, NG, G, CMAX>;
-  const unsigned FULL = 0xffffffffu;
-  const int wq = threadIdx.x & 31;
-  int total = 0, us = 0, bq = 0, gq = 0;
-  if (wq < ncomp) {
-    const int sl = wq / p.wpc;                         // chain slot of the warp
-    const int cq = chain0 + sl;
-    us = first_strip + (wq - sl * p.wpc);              // its strip, in scan order
-    if (cq < p.n_chains && us < p.strips) {
-      total = U;
-      bq = cq / p.n_cgroups;
-      gq = cq - bq * p.n_cgroups;
-    }
-  }
-  const uint32_t full0 = smem_u32(tfull + wq * kDepth);
-  const uint32_t empty0 = smem_u32(tempty + wq * kDepth);
-  unsigned char* ring = tiles0 + wq * DEPTH * L::TILE_BYTES;
-  int uu = 0, oi = 0, r = 0;                           // next row, as (orientation, scan row)
-  unsigned idle = 0;
-  long long t_idle = 0;
-  while (!__all_sync(FULL, uu >= total)) {
-    bool progressed = false;
-    if (uu < total) {
-      const int s = uu & (DEPTH - 1);
-      if (uu < DEPTH || mbar_test_wait(empty0 + s * 8, static_cast<unsigned>(((uu / DEPTH) - 1) & 1))) {
-        const int o = p.orient_code[oi];
-        const int i = (o & 2) ? p.H - 1 - r : r;           // stored row
-        const int t = (o & 1) ? p.strips - 1 - us : us;    // stored strip
-        const int k = p.orient_k[oi];
-        unsigned char* dst = ring + s * L::TILE_BYTES;
-        uint64_t* bar = tfull + wq * kDepth + s;
-        mbar_expect_tx(bar, L::TX_BYTES);
-        tma_load_4d(dst + L::X_OFF * L::ESZ, &tm.x, bar, t * CMAX, i, gq * L::CPW, bq);
-        tma_load_4d(dst + L::D_OFF * L::ESZ, &tm.d, bar, t * CMAX, i, gq * L::CPW, bq);
-        tma_load_4d(dst + L::B_OFF * L::ESZ, &tm.b, bar, t * CMAX, i, 0, bq * p.K + k);
-        tma_load_4d(dst + L::C_OFF * L::ESZ, &tm.c, bar, t * CMAX, i, 0, bq * p.K + k);
-        ++uu;
-        if (++r == p.H) { r = 0; ++oi; }
-        progressed = true;
-      }
-    }
-    (void)full0;
-    if (__any_sync(FULL, progressed)) {
-      idle = 0;
-    } else {
-      // nothing to stage right now: step aside for the compute warps, and give up (on every
-      // lane together) if no slot has freed up for the time limit
-      __nanosleep(32);
-      if (++idle == 1) t_idle = global_ns();
-      const bool late = (idle & 255u) == 0u && global_ns() - t_idle > p.timeout_ns;
-      if (__any_sync(FULL, late)) {
-        if (wq == 0) {
-          report_timeout(p.ctrl, p.gen);
-          *abort_flag = 1;
-        }
-        break;
-      }
-    }
-  }
-  if (wq < ncomp) issued[wq] = uu;
-}
-
 // ---- the kernel ------------------------------------------------------------------------------
 template <typename Tin, int NG, int G, int CMAX, bool TMA>
-__global__ void __launch_bounds__((kMaxWarps + 1) * 32)
+__global__ void __launch_bounds__(kMaxWarps * 32)
 scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps tm) {
   using L = Layout<Tin, NG, G, CMAX>;
   constexpr int PV = Elem<Tin>::kPerVec;
@@ -443,16 +403,14 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
 
   extern __shared__ __align__(1024) unsigned char smem[];
   __shared__ uint64_t s_tfull[kMaxWarps][kDepth];            // staged row landed (TMA)
-  __shared__ uint64_t s_tempty[kMaxWarps][kDepth];           // staged row consumed
   __shared__ uint64_t s_full[kMaxWarps][kCarryRing];         // carry slot written (consumer side)
   __shared__ uint64_t s_empty[kMaxWarps][kCarryRing];        // carry slot read (producer side)
   __shared__ int s_item;
-  __shared__ int s_abort;
 
   const unsigned FULL = 0xffffffffu;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  // compute warps 0 .. ncomp-1; with TMA one more warp issues every copy of the block
+  // every warp computes (and stages its own rows)
   const int ncomp = p.wpc * p.chains_per_block;
   const bool is_compute = warp < ncomp;
   const int slot = is_compute ? warp / p.wpc : 0;            // chain slot inside the block
@@ -464,7 +422,6 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
 
   // ---- which chain and segment -------------------------------------------------------
   if (threadIdx.x == 0) {
-    s_abort = 0;
     if (global_link) s_item = static_cast<int>(atomicAdd(&p.ctrl[0], 1ull));
   }
   __syncthreads();
@@ -521,15 +478,18 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   if (lane == 0 && is_compute) {
 #pragma unroll
     for (int s = 0; s < DEPTH; ++s) {
-      mbar_init(&s_tfull[warp][s], 1);        // the producer's expect_tx arrival + the bytes
-      mbar_init(&s_tempty[warp][s], 32);      // every lane of the compute warp
+      mbar_init(&s_tfull[warp][s], 1);        // lane 0's expect_tx arrival + the bytes
     }
 #pragma unroll
     for (int s = 0; s < kCarryRing; ++s) {
-      mbar_init(&s_full[warp][s], 32);
+      // a carry from another block arrives by st.async: this warp arms the slot itself
+      mbar_init(&s_full[warp][s], left_remote ? 1 : 32);
       mbar_init(&s_empty[warp][s], 32);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (left_remote)
+#pragma unroll
+      for (int s = 0; s < kCarryRing; ++s) mbar_arm_tx(smem_u32(&s_full[warp][s]), L::CARRY_SLOT_BYTES);
   }
   if (cluster) cluster_sync();      // every block's barriers exist before any remote arrive
   else __syncthreads();
@@ -596,13 +556,27 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   bool aborted = false;
   if (!TMA && strip_ok) plain_load(0);
 
-  // ---- the TMA producer warp: stages rows for every compute warp, never blocking on one ----
-  __shared__ int s_issued[kMaxWarps];                        // rows staged per compute warp
-  if (TMA && !is_compute) {
-    const int first = seg * p.wpc;
-    const int c0 = chain_of(0);
-    produce_rows<Tin, NG, G, CMAX, DEPTH>(p, tm, tiles0, &s_tfull[0][0], &s_tempty[0][0], s_issued, &s_abort,
-                                          ncomp, first, c0, U);
+  // ---- TMA: lane 0 stages the rows of this warp's walk, DEPTH rows ahead --------------------
+  // Row uu goes to slot uu % DEPTH; the warp refills a slot right after all its lanes have
+  // read it.  Once a wait of this warp has given up, nothing more is staged.
+  int staged = 0;                                            // rows of the walk staged so far
+  auto stage_row = [&](int uu) {                             // lane 0 only
+    int oi, i, t;
+    row_coords(uu, oi, i, t);
+    const int k = p.orient_k[oi];
+    const int s = uu % DEPTH;
+    unsigned char* dst = tiles + s * L::TILE_BYTES;
+    uint64_t* bar = &s_tfull[warp][s];
+    mbar_arm_tx(smem_u32(bar), L::TX_BYTES);
+    tma_load_4d(dst + L::X_OFF * L::ESZ, &tm.x, bar, t * CMAX, i, grp * L::CPW, b);
+    tma_load_4d(dst + L::D_OFF * L::ESZ, &tm.d, bar, t * CMAX, i, grp * L::CPW, b);
+    tma_load_4d(dst + L::B_OFF * L::ESZ, &tm.b, bar, t * CMAX, i, 0, b * p.K + k);
+    tma_load_4d(dst + L::C_OFF * L::ESZ, &tm.c, bar, t * CMAX, i, 0, b * p.K + k);
+  };
+  if (TMA && strip_ok) {
+    staged = U < DEPTH ? U : DEPTH;
+    if (lane == 0)
+      for (int uu = 0; uu < staged; ++uu) stage_row(uu);
   }
 
   // where this warp's carries go: the next warp of this block, or warp 0 of the next block
@@ -616,6 +590,38 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
     }
     if (left_remote) prev_empty_cl = map_rank(smem_u32(&s_empty[p.wpc - 1][0]), seg - 1);
   }
+
+  // global ring, consumer side: this lane's tagged words of the row it will need next
+  unsigned long long cw[L::CARRY2];
+  auto cw_load = [&](int uu) {
+    const unsigned long long* src =
+        p.carry + ((static_cast<size_t>(item - 1) * kRing + (uu % kRing)) * 32 + lane) * L::CARRY2;
+#pragma unroll
+    for (int k = 0; k < L::CARRY2 / 2; ++k) ld_relaxed_v2(src + 2 * k, cw[2 * k], cw[2 * k + 1]);
+  };
+  auto cw_ready = [&](unsigned want) {
+    bool ok = true;
+#pragma unroll
+    for (int e = 0; e < L::CARRY; ++e) ok = ok && static_cast<unsigned>(cw[e] >> 32) == want;
+    return ok;
+  };
+  // reloads row uu until every tag is right; true if it gave up (time-out or aborted launch)
+  auto cw_poll = [&](int uu) -> bool {
+    const unsigned want = ctag(p.gen, uu);
+    const long long t0 = global_ns();
+    for (unsigned it = 1;; ++it) {
+      if (cw_ready(want)) return false;
+      __nanosleep(32);
+      if ((it & 15u) == 0u) {
+        if (ld_acquire(&p.ctrl[2]) == p.gen) return true;
+        if (global_ns() - t0 > p.timeout_ns || it > (1u << 26)) {
+          report_timeout(p.ctrl, p.gen);
+          return true;
+        }
+      }
+      cw_load(uu);
+    }
+  };
 
   int u = 0;                                                 // rows of the walk done so far
   for (int oi = 0; oi < p.orient_count; ++oi) {
@@ -632,6 +638,15 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
       for (int c = 0; c < G; ++c)
 #pragma unroll
         for (int g = 0; g < NG; ++g) v[pp][c][g] = make_float2(0.f, 0.f);
+
+    if (left_global && strip_ok) {
+      // start two rows behind the upstream block, so that the words of the next row are
+      // already published when this warp requests them one row ahead
+      const int u1 = u + 1 < U ? u + 1 : u;
+      cw_load(u1);
+      if (!aborted) aborted = cw_poll(u1);
+      cw_load(u);
+    }
 
     for (int r = 0; r < H && strip_ok; ++r, ++u) {
       const int i = flipH ? H - 1 - r : r;
@@ -655,15 +670,13 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
       // ---- (2) carry-in: hh at the column before this strip (scan order) ----------------
       float hh[G][NG];
       if (left_global) {
-        const unsigned long long want = tag(p.gen, r + 1);
-        if (lane == 0) wait_geq(&p.flags[item - 1], want, p.ctrl, p.gen, p.timeout_ns);
-        __syncwarp();
-        const bool ok = ld_acquire(&p.flags[item - 1]) >= want;   // every lane acquires
-        const float* src = p.carry + ((static_cast<size_t>(item - 1) * kRing + (r % kRing)) * 32 + lane) * L::CARRY;
+        // this row's words were requested one row ago; every tag must be this row's
+        if (!aborted) aborted = cw_poll(u);
 #pragma unroll
         for (int c = 0; c < G; ++c)
 #pragma unroll
-          for (int g = 0; g < NG; ++g) hh[c][g] = ok ? __ldcg(src + c * NG + g) : 0.f;
+          for (int g = 0; g < NG; ++g) hh[c][g] = __uint_as_float(static_cast<unsigned>(cw[c * NG + g]));
+        if (u + 1 < U) cw_load(u + 1);
       } else if (has_left) {
         aborted = mbar_wait(smem_u32(&s_full[warp][cs]), cpar, p.ctrl, p.gen, p.timeout_ns, aborted);
         const float4* src = reinterpret_cast<const float4*>(carry_slot(warp, cs)) + lane * (L::CARRY_PAD / 4);
@@ -680,9 +693,8 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
         for (int c = 0; c < G; ++c)
 #pragma unroll
           for (int g = 0; g < NG; ++g) hh[c][g] = in[c * NG + g];
-        // free the slot: the producer waits on its own empty barrier
-        if (left_remote) mbar_arrive_remote(prev_empty_cl + cs * 8);
-        else mbar_arrive_local(smem_u32(&s_empty[warp - 1][cs]));
+        // free the slot (a slot filled from another block is freed once its values are used)
+        if (!left_remote) mbar_arrive_local(smem_u32(&s_empty[warp - 1][cs]));
       } else {
 #pragma unroll
         for (int c = 0; c < G; ++c)
@@ -745,8 +757,21 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
       }
 
       // ---- (4) the tile slot is free again: tell the producer warp (every lane has read) ------
-      if (TMA) mbar_arrive_local(smem_u32(&s_tempty[warp][s]));
-      else __syncwarp();
+      __syncwarp();
+      if (TMA && !aborted && staged < U) {
+        // every lane has read slot s: order those reads before the copy that refills it
+        if (lane == 0) {
+          fence_proxy_async();
+          stage_row(staged);
+        }
+        ++staged;
+      }
+      // a carry slot filled by the previous block: re-arm it for its next use, then free it;
+      // both are relaxed, so they never wait for this warp's outstanding stores of y
+      if (left_remote) {
+        if (lane == 0) mbar_arm_tx(smem_u32(&s_full[warp][cs]), L::CARRY_SLOT_BYTES);
+        mbar_arrive_remote_relaxed(prev_empty_cl + cs * 8);
+      }
 
       // ---- (5) carry-out to the next strip ---------------------------------------------------
       if (next_local || (next_remote && cluster)) {
@@ -767,33 +792,38 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
             dst[k4] = make_float4(out[4 * k4], out[4 * k4 + 1], out[4 * k4 + 2], out[4 * k4 + 3]);
           mbar_arrive_local(next_full0 + cs * 8);
         } else {
+          // st.async into the next block's slot: the bytes complete its full barrier
           const uint32_t dst = next_ring_cl + cs * L::CARRY_SLOT_BYTES + lane * L::CARRY_PAD * 4;
 #pragma unroll
           for (int k4 = 0; k4 < L::CARRY_PAD / 4; ++k4)
-            st_cluster_v4(dst + 16 * k4, out[4 * k4], out[4 * k4 + 1], out[4 * k4 + 2], out[4 * k4 + 3]);
-          mbar_arrive_remote(next_full_cl + cs * 8);
+            st_async_v4(dst + 16 * k4, out[4 * k4], out[4 * k4 + 1], out[4 * k4 + 2], out[4 * k4 + 3],
+                        next_full_cl + cs * 8);
         }
       } else if (next_remote && global_link) {
-        if (r >= kRing && (r % kPublish) == 0) {
-          // rows up to r - kRing must have been consumed before their slots are reused
-          const unsigned long long want = tag(p.gen, r - kRing + kPublish);
+        if (u >= kRing && (u % kPublish) == 0) {
+          // rows up to u - kRing must have been consumed before their slots are reused
+          const unsigned long long want = tag(p.gen, u - kRing + kPublish);
           if (lane == 0) wait_geq(&p.acks[item + 1], want, p.ctrl, p.gen, p.timeout_ns);
           __syncwarp();
-          (void)ld_acquire(&p.acks[item + 1]);           // orders this lane's ring writes
         }
-        float* dst = p.carry + ((static_cast<size_t>(item) * kRing + (r % kRing)) * 32 + lane) * L::CARRY;
+        // tagged words, no fence: the consumer checks every word's tag
+        unsigned long long* dst = p.carry + ((static_cast<size_t>(item) * kRing + (u % kRing)) * 32 + lane) * L::CARRY2;
+        const unsigned long long t = static_cast<unsigned long long>(ctag(p.gen, u)) << 32;
+        float out[L::CARRY2];
+        out[L::CARRY2 - 1] = 0.f;
 #pragma unroll
         for (int c = 0; c < G; ++c)
 #pragma unroll
-          for (int g = 0; g < NG; ++g) __stcg(dst + c * NG + g, hh[c][g]);
-        if ((r + 1) % kPublish == 0 || r == H - 1) {
-          __threadfence();
-          __syncwarp();
-          if (lane == 0) st_release(&p.flags[item], tag(p.gen, r + 1));
-        }
+          for (int g = 0; g < NG; ++g) out[c * NG + g] = hh[c][g];
+#pragma unroll
+        for (int k = 0; k < L::CARRY2 / 2; ++k)
+          st_relaxed_v2(dst + 2 * k, t | __float_as_uint(out[2 * k]), t | __float_as_uint(out[2 * k + 1]));
       }
-      if (left_global && ((r + 1) % kPublish == 0 || r == H - 1))
-        st_release(&p.acks[item], tag(p.gen, r + 1));   // every lane: its loads are done
+      // consumed rows, every kPublish rows (the words read so far are in use already)
+      if (left_global && ((u + 1) % kPublish == 0 || u == U - 1)) {
+        __syncwarp();
+        if (lane == 0) st_relaxed(&p.acks[item], tag(p.gen, u + 1));
+      }
 
       // ---- (6) reduce over the 4 state groups; lane q keeps the q-th quarter ------------------
       // flat index e = c*CMAX + j (channel-major, j = stored column in the strip)
@@ -860,17 +890,14 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
     if (p.mode == kSmemMulti && is_compute)
       asm volatile("bar.sync 1, %0;" ::"r"(ncomp * 32) : "memory");
   }
-  if (aborted) s_abort = 1;
-  __syncthreads();
-
-  // ---- after a timed-out wait: let the copies still in flight land (bounded) ------------------
-  if (TMA && !is_compute && lane == 0 && s_abort) {
+  // ---- after a timed-out wait: let this warp's copies still in flight land (bounded) -------
+  if (TMA && aborted && lane == 0) {
     bool gave_up = false;
-    for (int wq = 0; wq < ncomp; ++wq)
-      for (int uu = s_issued[wq] - DEPTH < 0 ? 0 : s_issued[wq] - DEPTH; uu < s_issued[wq]; ++uu)
-        gave_up = mbar_wait(smem_u32(&s_tfull[wq][uu % DEPTH]), static_cast<unsigned>((uu / DEPTH) & 1),
-                            p.ctrl, p.gen, p.timeout_ns, gave_up);
+    for (int uu = staged - DEPTH < 0 ? 0 : staged - DEPTH; uu < staged; ++uu)
+      gave_up = mbar_wait(smem_u32(&s_tfull[warp][uu % DEPTH]), static_cast<unsigned>((uu / DEPTH) & 1),
+                          p.ctrl, p.gen, p.timeout_ns, gave_up);
   }
+  __syncthreads();
 
   // ---- kSmemMulti: write the accumulated maps of this block's chains --------------------------
   if (p.mode == kSmemMulti && chain_ok) {
