@@ -66,15 +66,18 @@ using KernelFn = void (*)(const Params, const TmaMaps);
 
 struct Variant {
   int ng, g, cmax;            // states per lane, channels per lane, strip width
-  size_t tile_bytes;          // one staged strip row
+  size_t tile_bytes_tma;      // one staged tile of kTileRows strip rows (TMA path)
+  size_t tile_bytes_plain;    // one staged strip row (plain-load path)
   size_t carry_slot_bytes;    // one carry row of a warp
   KernelFn fn_tma, fn_plain;
 };
 
 template <typename Tin, int NG, int G, int CMAX>
 Variant make_variant() {
-  using L = Layout<Tin, NG, G, CMAX>;
-  return Variant{NG, G, CMAX, static_cast<size_t>(L::TILE_BYTES), static_cast<size_t>(L::CARRY_SLOT_BYTES),
+  using LT = Layout<Tin, NG, G, CMAX, kTileRows>;
+  using LP = Layout<Tin, NG, G, CMAX, 1>;
+  return Variant{NG, G, CMAX, static_cast<size_t>(LT::TILE_BYTES), static_cast<size_t>(LP::TILE_BYTES),
+                 static_cast<size_t>(LP::CARRY_SLOT_BYTES),
                  scan2d_kernel<Tin, NG, G, CMAX, true>, scan2d_kernel<Tin, NG, G, CMAX, false>};
 }
 
@@ -135,7 +138,7 @@ Plan make_plan(const Shape& s, int ng, bool g1, bool tma) {
   }
   pl.warps = pl.wpc * pl.chains_per_block;
   pl.carry_smem = static_cast<size_t>(pl.warps) * kCarryRing * pl.var.carry_slot_bytes;
-  pl.tile_smem = static_cast<size_t>(pl.warps) * (tma ? kDepth : 1) * pl.var.tile_bytes;
+  pl.tile_smem = static_cast<size_t>(pl.warps) * (tma ? kTileDepth * pl.var.tile_bytes_tma : pl.var.tile_bytes_plain);
   return pl;
 }
 
@@ -159,18 +162,21 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 4-D map (W, H, d2, d3) of a dense tensor with a (cmax, 1, box2, 1) box.
+// 4-D map of a dense (d3, d2, H, W) tensor, with dimensions listed as (W, d2, H, d3), so that a
+// (cmax, box2, kTileRows, 1) box lands in shared memory as kTileRows consecutive [box2][cmax]
+// row tiles.
 bool encode_map(CUtensorMap* m, const void* base, bool bf16, int W, int H, long long d2,
                 long long d3, int cmax, int box2) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const size_t e = bf16 ? 2 : 4;
-  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(W), static_cast<cuuint64_t>(H),
-                              static_cast<cuuint64_t>(d2), static_cast<cuuint64_t>(d3)};
-  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(W) * e,
-                                 static_cast<cuuint64_t>(W) * H * e,
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(W), static_cast<cuuint64_t>(d2),
+                              static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(d3)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(W) * H * e,
+                                 static_cast<cuuint64_t>(W) * e,
                                  static_cast<cuuint64_t>(W) * H * e * d2};
-  const cuuint32_t box[4] = {static_cast<cuuint32_t>(cmax), 1u, static_cast<cuuint32_t>(box2), 1u};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(cmax), static_cast<cuuint32_t>(box2),
+                             static_cast<cuuint32_t>(kTileRows), 1u};
   const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
   const CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
                         const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,

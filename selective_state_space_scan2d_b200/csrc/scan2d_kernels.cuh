@@ -54,7 +54,8 @@ constexpr int kGroups = 8;             // channel groups per warp
 constexpr int kRing = 16;              // carry rows buffered in global memory between blocks
 constexpr int kCarryRing = 4;          // carry rows buffered in shared memory between warps
 constexpr int kMaxWarps = 8;           // compute warps per block (plus one TMA producer warp)
-constexpr int kDepth = 4;              // rows staged ahead per warp (TMA path)
+constexpr int kTileRows = 4;           // rows per staged tile (TMA path; the plain path stages 1)
+constexpr int kTileDepth = 2;          // staged tiles in flight per warp (TMA path)
 constexpr int kPublish = 4;            // global fallback: rows per flag release
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -213,24 +214,15 @@ __device__ __forceinline__ void st_async_v4(uint32_t addr, float a, float b, flo
                : "memory");
 }
 
+// One try of phase `parity` of an mbarrier of this block; true once the phase has completed.
+// CTA scope: every mbarrier waited on is this block's own, and the data it guards arrives
+// either by this block's stores (release.cta arrives), by TMA or by st.async (both signalled
+// through the barrier's transaction count).
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, unsigned parity) {
   unsigned ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Non-blocking test of phase `parity` of an mbarrier.
-__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, unsigned parity) {
-  unsigned ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
@@ -245,10 +237,6 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
       " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
       : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // Records a device error once and marks this launch generation aborted: every other wait of
@@ -353,22 +341,25 @@ __device__ __forceinline__ void store_out4(void* y, size_t idx, const float* v, 
 }
 
 // ---- shared memory of one block ---------------------------------------------------------------
-template <typename Tin, int NG, int G, int CMAX>
+template <typename Tin, int NG, int G, int CMAX, int R = 1>
 struct Layout {
   static constexpr int ESZ = static_cast<int>(sizeof(Tin));
   static constexpr int CPW = kGroups * G;                    // channels per warp
   static constexpr int NB = kQ * NG;                         // states covered by the 4 q lanes
-  static constexpr int X_BYTES = CPW * CMAX * ESZ;           // [CPW][CMAX]
-  static constexpr int B_BYTES = NB * CMAX * ESZ;            // [NB][CMAX]
+  static constexpr int X_ROW = CPW * CMAX;                   // elements of one row: [CPW][CMAX]
+  static constexpr int B_ROW = NB * CMAX;                    // [NB][CMAX]
+  static constexpr int X_BYTES = R * X_ROW * ESZ;            // R rows: [R][CPW][CMAX]
+  static constexpr int B_BYTES = R * B_ROW * ESZ;            // [R][NB][CMAX]
   static constexpr int r128(int v) { return (v + 127) / 128 * 128; }
-  // one staged strip row; every region starts on a 128-byte boundary (TMA destinations)
+  // one staged tile of R strip rows; every region starts on a 128-byte boundary (TMA
+  // destinations)
   static constexpr int X_OFF = 0;                                        // element offsets
   static constexpr int D_OFF = r128(X_BYTES) / ESZ;
   static constexpr int B_OFF = D_OFF + r128(X_BYTES) / ESZ;
   static constexpr int C_OFF = B_OFF + r128(B_BYTES) / ESZ;
   static constexpr int TILE_BYTES = (C_OFF * ESZ) + r128(B_BYTES);
   static constexpr int TX_BYTES = 2 * X_BYTES + 2 * B_BYTES;
-  static constexpr int DENSE = (2 * CPW + 2 * NB) * CMAX;    // tile values without padding
+  static constexpr int DENSE = (2 * CPW + 2 * NB) * CMAX;    // values of one row without padding
   static constexpr int PLAIN_PER_LANE = DENSE / 32;          // plain-load path: values per lane
   static constexpr int CARRY = G * NG;                       // carry floats per lane
   static constexpr int CARRY_PAD = (CARRY + 3) / 4 * 4;      // ... padded to whole float4s
@@ -391,18 +382,19 @@ __host__ __device__ constexpr size_t carry_ring_bytes(int warps) {
 template <typename Tin, int NG, int G, int CMAX, bool TMA>
 __global__ void __launch_bounds__(kMaxWarps * 32)
 scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps tm) {
-  using L = Layout<Tin, NG, G, CMAX>;
+  constexpr int R = TMA ? kTileRows : 1;                     // rows per staged tile
+  using L = Layout<Tin, NG, G, CMAX, R>;
   constexpr int PV = Elem<Tin>::kPerVec;
   static_assert(CMAX % PV == 0, "strip width must hold whole 16-byte vectors");
   static_assert(L::E % 4 == 0, "reduce-scatter needs 4 | CMAX*G");
   static_assert(L::DENSE % 32 == 0, "plain-load path needs 32 | tile values");
-  constexpr int DEPTH = TMA ? kDepth : 1;
+  constexpr int DEPTH = TMA ? kTileDepth : 1;
   constexpr int NVEC = CMAX / PV;                            // 16-byte vectors per strip row
   constexpr int E = L::E;
   constexpr int NP = L::NP;
 
   extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ uint64_t s_tfull[kMaxWarps][kDepth];            // staged row landed (TMA)
+  __shared__ uint64_t s_tfull[kMaxWarps][kTileDepth];        // staged tile landed (TMA)
   __shared__ uint64_t s_full[kMaxWarps][kCarryRing];         // carry slot written (consumer side)
   __shared__ uint64_t s_empty[kMaxWarps][kCarryRing];        // carry slot read (producer side)
   __shared__ int s_item;
@@ -556,27 +548,34 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   bool aborted = false;
   if (!TMA && strip_ok) plain_load(0);
 
-  // ---- TMA: lane 0 stages the rows of this warp's walk, DEPTH rows ahead --------------------
-  // Row uu goes to slot uu % DEPTH; the warp refills a slot right after all its lanes have
-  // read it.  Once a wait of this warp has given up, nothing more is staged.
-  int staged = 0;                                            // rows of the walk staged so far
-  auto stage_row = [&](int uu) {                             // lane 0 only
-    int oi, i, t;
-    row_coords(uu, oi, i, t);
+  // ---- TMA: lane 0 stages the tiles of this warp's walk, DEPTH tiles ahead -----------------
+  // A tile is R consecutive scan rows of one orientation (the last one may reach past the map:
+  // TMA fills those rows with zeros).  Walk tile wt goes to slot wt % DEPTH; the warp refills
+  // a slot right after all its lanes have read the tile's last row.  Once a wait of this warp
+  // has given up, nothing more is staged.
+  const int TPO = (H + R - 1) / R;                           // tiles per orientation
+  const int UT = p.orient_count * TPO;                       // tiles of the walk
+  int staged = 0;                                            // tiles of the walk staged so far
+  auto stage_tile = [&](int wt) {                            // lane 0 only
+    const int oi = wt / TPO;
+    const int tr = wt - oi * TPO;
+    const int o = p.orient_code[oi];
+    const int row0 = (o & 2) ? H - R - tr * R : tr * R;      // first stored row of the box
+    const int t = (o & 1) ? p.strips - 1 - u_scan : u_scan;  // stored strip
     const int k = p.orient_k[oi];
-    const int s = uu % DEPTH;
+    const int s = wt % DEPTH;
     unsigned char* dst = tiles + s * L::TILE_BYTES;
     uint64_t* bar = &s_tfull[warp][s];
     mbar_arm_tx(smem_u32(bar), L::TX_BYTES);
-    tma_load_4d(dst + L::X_OFF * L::ESZ, &tm.x, bar, t * CMAX, i, grp * L::CPW, b);
-    tma_load_4d(dst + L::D_OFF * L::ESZ, &tm.d, bar, t * CMAX, i, grp * L::CPW, b);
-    tma_load_4d(dst + L::B_OFF * L::ESZ, &tm.b, bar, t * CMAX, i, 0, b * p.K + k);
-    tma_load_4d(dst + L::C_OFF * L::ESZ, &tm.c, bar, t * CMAX, i, 0, b * p.K + k);
+    tma_load_4d(dst + L::X_OFF * L::ESZ, &tm.x, bar, t * CMAX, grp * L::CPW, row0, b);
+    tma_load_4d(dst + L::D_OFF * L::ESZ, &tm.d, bar, t * CMAX, grp * L::CPW, row0, b);
+    tma_load_4d(dst + L::B_OFF * L::ESZ, &tm.b, bar, t * CMAX, 0, row0, b * p.K + k);
+    tma_load_4d(dst + L::C_OFF * L::ESZ, &tm.c, bar, t * CMAX, 0, row0, b * p.K + k);
   };
   if (TMA && strip_ok) {
-    staged = U < DEPTH ? U : DEPTH;
+    staged = UT < DEPTH ? UT : DEPTH;
     if (lane == 0)
-      for (int uu = 0; uu < staged; ++uu) stage_row(uu);
+      for (int wt = 0; wt < staged; ++wt) stage_tile(wt);
   }
 
   // where this warp's carries go: the next warp of this block, or warp 0 of the next block
@@ -650,15 +649,19 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
 
     for (int r = 0; r < H && strip_ok; ++r, ++u) {
       const int i = flipH ? H - 1 - r : r;
-      const int s = u % DEPTH;
+      const int tr = r / R, rr = r - tr * R;                 // tile of the orientation, row in it
+      const int wt = oi * TPO + tr;                          // tile of the walk
+      const int s = wt % DEPTH;
+      const int rt = flipH ? R - 1 - rr : rr;                // this row's place in the staged tile
       const Tin* tile = reinterpret_cast<const Tin*>(tiles + s * L::TILE_BYTES);
       const int cs = u % kCarryRing;                         // carry ring slot of this row
       const unsigned cpar = static_cast<unsigned>((u / kCarryRing) & 1);
 
       // ---- (1) this row's tile is in shared memory -----------------------------------
       if (TMA) {
-        aborted = mbar_wait(smem_u32(&s_tfull[warp][s]), static_cast<unsigned>((u / DEPTH) & 1), p.ctrl,
-                            p.gen, p.timeout_ns, aborted);
+        if (rr == 0)
+          aborted = mbar_wait(smem_u32(&s_tfull[warp][s]), static_cast<unsigned>((wt / DEPTH) & 1), p.ctrl,
+                              p.gen, p.timeout_ns, aborted);
       } else {
         Tin* dst = reinterpret_cast<Tin*>(tiles);
 #pragma unroll
@@ -708,13 +711,13 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
         uint4 xv[G], dv[G], bv[NG], cv[NG];
 #pragma unroll
         for (int c = 0; c < G; ++c) {
-          xv[c] = *reinterpret_cast<const uint4*>(tile + L::X_OFF + (cg * G + c) * CMAX + vg * PV);
-          dv[c] = *reinterpret_cast<const uint4*>(tile + L::D_OFF + (cg * G + c) * CMAX + vg * PV);
+          xv[c] = *reinterpret_cast<const uint4*>(tile + L::X_OFF + rt * L::X_ROW + (cg * G + c) * CMAX + vg * PV);
+          dv[c] = *reinterpret_cast<const uint4*>(tile + L::D_OFF + rt * L::X_ROW + (cg * G + c) * CMAX + vg * PV);
         }
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
-          bv[g] = *reinterpret_cast<const uint4*>(tile + L::B_OFF + (q + kQ * g) * CMAX + vg * PV);
-          cv[g] = *reinterpret_cast<const uint4*>(tile + L::C_OFF + (q + kQ * g) * CMAX + vg * PV);
+          bv[g] = *reinterpret_cast<const uint4*>(tile + L::B_OFF + rt * L::B_ROW + (q + kQ * g) * CMAX + vg * PV);
+          cv[g] = *reinterpret_cast<const uint4*>(tile + L::C_OFF + rt * L::B_ROW + (q + kQ * g) * CMAX + vg * PV);
         }
 #pragma unroll
         for (int k = 0; k < PV / 2; ++k) {
@@ -758,12 +761,9 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
 
       // ---- (4) the tile slot is free again: tell the producer warp (every lane has read) ------
       __syncwarp();
-      if (TMA && !aborted && staged < U) {
-        // every lane has read slot s: order those reads before the copy that refills it
-        if (lane == 0) {
-          fence_proxy_async();
-          stage_row(staged);
-        }
+      if (TMA && (rr == R - 1 || r == H - 1) && !aborted && staged < UT) {
+        // every lane has read the tile's last row (its values are in use): refill the slot
+        if (lane == 0) stage_tile(staged);
         ++staged;
       }
       // a carry slot filled by the previous block: re-arm it for its next use, then free it;
@@ -893,8 +893,8 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   // ---- after a timed-out wait: let this warp's copies still in flight land (bounded) -------
   if (TMA && aborted && lane == 0) {
     bool gave_up = false;
-    for (int uu = staged - DEPTH < 0 ? 0 : staged - DEPTH; uu < staged; ++uu)
-      gave_up = mbar_wait(smem_u32(&s_tfull[warp][uu % DEPTH]), static_cast<unsigned>((uu / DEPTH) & 1),
+    for (int wt = staged - DEPTH < 0 ? 0 : staged - DEPTH; wt < staged; ++wt)
+      gave_up = mbar_wait(smem_u32(&s_tfull[warp][wt % DEPTH]), static_cast<unsigned>((wt / DEPTH) & 1),
                           p.ctrl, p.gen, p.timeout_ns, gave_up);
   }
   __syncthreads();
