@@ -75,6 +75,23 @@ def base_config(w: inputs.Workload, world: int) -> dict:
             "global_batch": w.batch * world, "parallelism": f"replicas x{world}"}
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise max of per-rank values over all ranks (the values themselves without a
+    process group); every rank calls it with the same number of values."""
+    import torch
+    if not torch.distributed.is_initialized() or torch.distributed.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def whole_job_gelem(elements_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job throughput: every rank processes its own instance of the workload (weak
+    scaling), timed by the slowest rank."""
+    return world * elements_per_rank / (ms * 1e-3) / 1e9
+
+
 KERNEL_SOURCES = ("selective_state_space_scan2d_b200/csrc/scan2d.cu",
                   "selective_state_space_scan2d_b200/csrc/scan2d_kernels.cuh")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "scan2d_dram_traffic.txt")
@@ -352,12 +369,9 @@ def main():
                            warmup=args.warmup, with_e2e=not args.no_e2e)
     ms = res["ms"]
     e2e_ms = res["e2e"]["ms"] if "e2e" in res else float("nan")
-    if world > 1:
-        t = torch.tensor([ms, e2e_ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, e2e_ms = float(t[0]), float(t[1])
-    value = world * w.elements / (ms * 1e-3) / 1e9
-    e2e_value = world * w.elements / (e2e_ms * 1e-3) / 1e9
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], device=device)
+    value = whole_job_gelem(w.elements, world, ms)
+    e2e_value = whole_job_gelem(w.elements, world, e2e_ms)
 
     rm = roofline_model(w)
     if rm["bound"] == "sfu":
