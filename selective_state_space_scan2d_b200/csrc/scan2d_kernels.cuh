@@ -148,6 +148,12 @@ __device__ __forceinline__ unsigned ctag(unsigned long long gen, int r) {
   return (static_cast<unsigned>(gen & 0xFFFFFull) << 12) | (static_cast<unsigned>(r + 1) & 0xFFFu);
 }
 
+__device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
 __device__ __forceinline__ void st_relaxed(unsigned long long* p, unsigned long long v) {
   asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
@@ -622,6 +628,7 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
     }
   };
 
+  unsigned long long ack_seen = 0;                           // global ring: last ack read
   int u = 0;                                                 // rows of the walk done so far
   for (int oi = 0; oi < p.orient_count; ++oi) {
     const int o = p.orient_code[oi];
@@ -759,21 +766,7 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
         for (int vg = NVEC - 1; vg >= 0; --vg) vec_group(vg, true);
       }
 
-      // ---- (4) the tile slot is free again: tell the producer warp (every lane has read) ------
-      __syncwarp();
-      if (TMA && (rr == R - 1 || r == H - 1) && !aborted && staged < UT) {
-        // every lane has read the tile's last row (its values are in use): refill the slot
-        if (lane == 0) stage_tile(staged);
-        ++staged;
-      }
-      // a carry slot filled by the previous block: re-arm it for its next use, then free it;
-      // both are relaxed, so they never wait for this warp's outstanding stores of y
-      if (left_remote) {
-        if (lane == 0) mbar_arm_tx(smem_u32(&s_full[warp][cs]), L::CARRY_SLOT_BYTES);
-        mbar_arrive_remote_relaxed(prev_empty_cl + cs * 8);
-      }
-
-      // ---- (5) carry-out to the next strip ---------------------------------------------------
+      // ---- (4) carry-out to the next strip, as early as possible -----------------------------
       if (next_local || (next_remote && cluster)) {
         // the slot is free once the consumer released its previous use
         if (u >= kCarryRing)
@@ -801,10 +794,14 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
         }
       } else if (next_remote && global_link) {
         if (u >= kRing && (u % kPublish) == 0) {
-          // rows up to u - kRing must have been consumed before their slots are reused
+          // rows up to u - kRing must have been consumed before their slots are reused; the
+          // ack read kPublish rows ago usually shows that already, else wait for it (bounded)
           const unsigned long long want = tag(p.gen, u - kRing + kPublish);
-          if (lane == 0) wait_geq(&p.acks[item + 1], want, p.ctrl, p.gen, p.timeout_ns);
-          __syncwarp();
+          if (ack_seen < want) {
+            if (lane == 0) wait_geq(&p.acks[item + 1], want, p.ctrl, p.gen, p.timeout_ns);
+            __syncwarp();
+          }
+          ack_seen = ld_relaxed(&p.acks[item + 1]);           // for the next check, not waited on
         }
         // tagged words, no fence: the consumer checks every word's tag
         unsigned long long* dst = p.carry + ((static_cast<size_t>(item) * kRing + (u % kRing)) * 32 + lane) * L::CARRY2;
@@ -823,6 +820,20 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
       if (left_global && ((u + 1) % kPublish == 0 || u == U - 1)) {
         __syncwarp();
         if (lane == 0) st_relaxed(&p.acks[item], tag(p.gen, u + 1));
+      }
+
+      // ---- (5) refill the tile slot (every lane has read the tile's last row) ---------------
+      __syncwarp();
+      if (TMA && (rr == R - 1 || r == H - 1) && !aborted && staged < UT) {
+        // every lane has read the tile's last row (its values are in use): refill the slot
+        if (lane == 0) stage_tile(staged);
+        ++staged;
+      }
+      // a carry slot filled by the previous block: re-arm it for its next use, then free it;
+      // both are relaxed, so they never wait for this warp's outstanding stores of y
+      if (left_remote) {
+        if (lane == 0) mbar_arm_tx(smem_u32(&s_full[warp][cs]), L::CARRY_SLOT_BYTES);
+        mbar_arrive_remote_relaxed(prev_empty_cl + cs * 8);
       }
 
       // ---- (6) reduce over the 4 state groups; lane q keeps the q-th quarter ------------------
