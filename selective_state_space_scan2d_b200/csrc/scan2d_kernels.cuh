@@ -386,7 +386,7 @@ __host__ __device__ constexpr size_t carry_ring_bytes(int warps) {
 
 // ---- the kernel ------------------------------------------------------------------------------
 template <typename Tin, int NG, int G, int CMAX, bool TMA>
-__global__ void __launch_bounds__(kMaxWarps * 32)
+__global__ void __launch_bounds__(kMaxWarps * 32, 1)
 scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps tm) {
   constexpr int R = TMA ? kTileRows : 1;                     // rows per staged tile
   using L = Layout<Tin, NG, G, CMAX, R>;
@@ -562,26 +562,37 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   const int TPO = (H + R - 1) / R;                           // tiles per orientation
   const int UT = p.orient_count * TPO;                       // tiles of the walk
   int staged = 0;                                            // tiles of the walk staged so far
-  auto stage_tile = [&](int wt) {                            // lane 0 only
-    const int oi = wt / TPO;
-    const int tr = wt - oi * TPO;
-    const int o = p.orient_code[oi];
-    const int row0 = (o & 2) ? H - R - tr * R : tr * R;      // first stored row of the box
-    const int t = (o & 1) ? p.strips - 1 - u_scan : u_scan;  // stored strip
-    const int k = p.orient_k[oi];
-    const int s = wt % DEPTH;
+  // the next tile to stage, as (orientation, tile in it), with that orientation's stored strip
+  // column, flip and B/C index (lane 0's copy is the one in use)
+  int st_oi = 0, st_tr = 0, st_col = 0, st_flip = 0, st_bk = 0;
+  auto st_orientation = [&]() {
+    const int o = p.orient_code[st_oi];
+    st_flip = o & 2;
+    st_col = ((o & 1) ? p.strips - 1 - u_scan : u_scan) * CMAX;
+    st_bk = b * p.K + p.orient_k[st_oi];
+  };
+  auto stage_tile = [&]() {                                  // lane 0 only: walk tile `staged`
+    const int row0 = st_flip ? H - R - st_tr * R : st_tr * R;  // first stored row of the box
+    const int s = staged % DEPTH;
     unsigned char* dst = tiles + s * L::TILE_BYTES;
     uint64_t* bar = &s_tfull[warp][s];
     mbar_arm_tx(smem_u32(bar), L::TX_BYTES);
-    tma_load_4d(dst + L::X_OFF * L::ESZ, &tm.x, bar, t * CMAX, grp * L::CPW, row0, b);
-    tma_load_4d(dst + L::D_OFF * L::ESZ, &tm.d, bar, t * CMAX, grp * L::CPW, row0, b);
-    tma_load_4d(dst + L::B_OFF * L::ESZ, &tm.b, bar, t * CMAX, 0, row0, b * p.K + k);
-    tma_load_4d(dst + L::C_OFF * L::ESZ, &tm.c, bar, t * CMAX, 0, row0, b * p.K + k);
+    tma_load_4d(dst + L::X_OFF * L::ESZ, &tm.x, bar, st_col, grp * L::CPW, row0, b);
+    tma_load_4d(dst + L::D_OFF * L::ESZ, &tm.d, bar, st_col, grp * L::CPW, row0, b);
+    tma_load_4d(dst + L::B_OFF * L::ESZ, &tm.b, bar, st_col, 0, row0, st_bk);
+    tma_load_4d(dst + L::C_OFF * L::ESZ, &tm.c, bar, st_col, 0, row0, st_bk);
+    if (++st_tr == TPO) {
+      st_tr = 0;
+      if (++st_oi < p.orient_count) st_orientation();
+    }
   };
   if (TMA && strip_ok) {
-    staged = UT < DEPTH ? UT : DEPTH;
-    if (lane == 0)
-      for (int wt = 0; wt < staged; ++wt) stage_tile(wt);
+    const int first = UT < DEPTH ? UT : DEPTH;
+    if (lane == 0) {
+      st_orientation();
+      for (; staged < first; ++staged) stage_tile();
+    }
+    staged = first;
   }
 
   // where this warp's carries go: the next warp of this block, or warp 0 of the next block
@@ -653,6 +664,74 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
       if (!aborted) aborted = cw_poll(u1);
       cw_load(u);
     }
+
+    // row outputs are written one row late: the reduction of row r over the 4 state-group
+    // lanes is issued together with the math of row r + 1, so the two overlap
+    float2 pacc[NP][G];                                      // partial outputs of the pending row
+#pragma unroll
+    for (int pp = 0; pp < NP; ++pp)
+#pragma unroll
+      for (int c = 0; c < G; ++c) pacc[pp][c] = make_float2(0.f, 0.f);
+    int p_i = -1;                                            // stored row of the pending row
+
+    // reduce-scatter over the 4 state-group lanes of a channel group: lane q keeps the q-th
+    // quarter of the flat index e = c*CMAX + j (channel-major, j = stored column in the strip)
+    auto reduce_row = [&](const float2 (&ac)[NP][G], float (&own)[E / 4]) {
+      float flat[E];
+#pragma unroll
+      for (int c = 0; c < G; ++c)
+#pragma unroll
+        for (int pp = 0; pp < NP; ++pp) {
+          flat[c * CMAX + 2 * pp] = ac[pp][c].x;
+          flat[c * CMAX + 2 * pp + 1] = ac[pp][c].y;
+        }
+      float r1[E / 2];
+      const bool hi2 = (q & 2) != 0, hi1 = (q & 1) != 0;
+#pragma unroll
+      for (int e = 0; e < E / 2; ++e) {
+        const float lo = flat[e], hi = flat[e + E / 2];
+        r1[e] = (hi2 ? hi : lo) + __shfl_xor_sync(FULL, hi2 ? lo : hi, 2);
+      }
+#pragma unroll
+      for (int e = 0; e < E / 4; ++e) {
+        const float lo = r1[e], hi = r1[e + E / 4];
+        own[e] = (hi1 ? hi : lo) + __shfl_xor_sync(FULL, hi1 ? lo : hi, 1);
+      }
+    };
+    // output of stored row i_row: channel c, columns j0 .. j0 + E/4 - 1 of the strip
+    auto write_row = [&](int i_row, const float (&own)[E / 4]) {
+      const int e0 = q * (E / 4);
+      const int c = e0 / CMAX;
+      const int j0 = e0 - c * CMAX;
+      const int d = ch0 + c;
+      if (d >= p.channels) return;
+      const size_t rowoff = (static_cast<size_t>(b) * p.channels + d) * HW + static_cast<size_t>(i_row) * W;
+      const int gc = col0 + j0;
+      if (p.mode == kSingle) {
+        if ((E / 4) % 4 == 0 && p.vec_store && gc + E / 4 <= W) {
+#pragma unroll
+          for (int m = 0; m < E / 4; m += 4) store_out4(p.y, rowoff + gc + m, own + m, p.out_f32);
+        } else {
+#pragma unroll
+          for (int m = 0; m < E / 4; ++m)
+            if (gc + m < W) store_out(p.y, rowoff + gc + m, own[m], p.out_f32);
+        }
+      } else if (p.mode == kSmemMulti) {
+        float* a = yacc_s + (slot * L::CPW + cg * G + c) * p.yacc_stride + i_row * W + gc;
+#pragma unroll
+        for (int m = 0; m < E / 4; ++m)
+          if (gc + m < W) a[m] = (oi == 0) ? own[m] : a[m] + own[m];
+      } else {
+#pragma unroll
+        for (int m = 0; m < E / 4; ++m) {
+          if (gc + m >= W) continue;
+          const size_t idx = rowoff + gc + m;
+          if (p.mode == kGlobalFirst) p.yacc[idx] = own[m];
+          else if (p.mode == kGlobalMid) p.yacc[idx] += own[m];
+          else store_out(p.y, idx, p.yacc[idx] + own[m], p.out_f32);
+        }
+      }
+    };
 
     for (int r = 0; r < H && strip_ok; ++r, ++u) {
       const int i = flipH ? H - 1 - r : r;
@@ -758,10 +837,13 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
           }
         }
       };
+      float own_prev[E / 4];                                 // the pending row, reduced
       if (!flipW) {
+        reduce_row(pacc, own_prev);
 #pragma unroll
         for (int vg = 0; vg < NVEC; ++vg) vec_group(vg, false);
       } else {
+        reduce_row(pacc, own_prev);
 #pragma unroll
         for (int vg = NVEC - 1; vg >= 0; --vg) vec_group(vg, true);
       }
@@ -826,7 +908,7 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
       __syncwarp();
       if (TMA && (rr == R - 1 || r == H - 1) && !aborted && staged < UT) {
         // every lane has read the tile's last row (its values are in use): refill the slot
-        if (lane == 0) stage_tile(staged);
+        if (lane == 0) stage_tile();
         ++staged;
       }
       // a carry slot filled by the previous block: re-arm it for its next use, then free it;
@@ -836,65 +918,19 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
         mbar_arrive_remote_relaxed(prev_empty_cl + cs * 8);
       }
 
-      // ---- (6) reduce over the 4 state groups; lane q keeps the q-th quarter ------------------
-      // flat index e = c*CMAX + j (channel-major, j = stored column in the strip)
-      float flat[E];
+      // ---- (6) the previous row's output (its reduction was interleaved with this row's math) --
+      if (p_i >= 0) write_row(p_i, own_prev);
 #pragma unroll
-      for (int c = 0; c < G; ++c)
+      for (int pp = 0; pp < NP; ++pp)
 #pragma unroll
-        for (int pp = 0; pp < NP; ++pp) {
-          flat[c * CMAX + 2 * pp] = acc[pp][c].x;
-          flat[c * CMAX + 2 * pp + 1] = acc[pp][c].y;
-        }
-      float r1[E / 2];
-      const bool hi2 = (q & 2) != 0, hi1 = (q & 1) != 0;
-#pragma unroll
-      for (int e = 0; e < E / 2; ++e) {
-        const float lo = flat[e], hi = flat[e + E / 2];
-        r1[e] = (hi2 ? hi : lo) + __shfl_xor_sync(FULL, hi2 ? lo : hi, 2);
-      }
-      float own[E / 4];
-#pragma unroll
-      for (int e = 0; e < E / 4; ++e) {
-        const float lo = r1[e], hi = r1[e + E / 4];
-        own[e] = (hi1 ? hi : lo) + __shfl_xor_sync(FULL, hi1 ? lo : hi, 1);
-      }
-
-      // ---- (7) output: channel c, columns j0 .. j0 + E/4 - 1 of the strip --------------------
-      {
-        const int e0 = q * (E / 4);
-        const int c = e0 / CMAX;
-        const int j0 = e0 - c * CMAX;
-        const int d = ch0 + c;
-        if (d < p.channels) {
-          const size_t rowoff = (static_cast<size_t>(b) * p.channels + d) * HW + static_cast<size_t>(i) * W;
-          const int gc = col0 + j0;
-          if (p.mode == kSingle) {
-            if ((E / 4) % 4 == 0 && p.vec_store && gc + E / 4 <= W) {
-#pragma unroll
-              for (int m = 0; m < E / 4; m += 4) store_out4(p.y, rowoff + gc + m, own + m, p.out_f32);
-            } else {
-#pragma unroll
-              for (int m = 0; m < E / 4; ++m)
-                if (gc + m < W) store_out(p.y, rowoff + gc + m, own[m], p.out_f32);
-            }
-          } else if (p.mode == kSmemMulti) {
-            float* a = yacc_s + (slot * L::CPW + cg * G + c) * p.yacc_stride + i * W + gc;
-#pragma unroll
-            for (int m = 0; m < E / 4; ++m)
-              if (gc + m < W) a[m] = (oi == 0) ? own[m] : a[m] + own[m];
-          } else {
-#pragma unroll
-            for (int m = 0; m < E / 4; ++m) {
-              if (gc + m >= W) continue;
-              const size_t idx = rowoff + gc + m;
-              if (p.mode == kGlobalFirst) p.yacc[idx] = own[m];
-              else if (p.mode == kGlobalMid) p.yacc[idx] += own[m];
-              else store_out(p.y, idx, p.yacc[idx] + own[m], p.out_f32);
-            }
-          }
-        }
-      }
+        for (int c = 0; c < G; ++c) pacc[pp][c] = acc[pp][c];
+      p_i = i;
+    }
+    // the orientation's last row
+    if (p_i >= 0) {
+      float own_last[E / 4];
+      reduce_row(pacc, own_last);
+      write_row(p_i, own_last);
     }
     // orientations summed in shared memory: no compute warp may start the next orientation
     // (whose strips map to other columns) before every compute warp has finished this one
