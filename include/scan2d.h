@@ -126,8 +126,8 @@ int scan2d_fwd_noalloc(const void *x, const void *delta, const float *A, const v
                        int H, int W, int N, unsigned flags, void *stream);
 
 /*
- * scan2d_query_plan -- how scan2d_fwd would run a call of this shape, without launching
- * anything or touching a device.  Writes up to n_out (<= SCAN2D_PLAN_FIELDS) values to `out`:
+ * scan2d_query_plan -- how scan2d_fwd would run a call of this shape on a B200 (148
+ * multiprocessors, clusters assumed resident), without launching anything or touching a device.  Writes up to n_out (<= SCAN2D_PLAN_FIELDS) values to `out`:
  *   [0] kernel launches per call        [5] columns per warp strip
  *   [1] blocks per launch               [6] warps (strips) per chain in a block
  *   [2] threads per block               [7] 0 one orientation, 1 orientations summed in

@@ -266,7 +266,13 @@ struct CallPlan {
   size_t smem, items, carry_bytes, yacc_bytes, ws_bytes;
 };
 
-CallPlan plan_call(const Shape& s, bool tma, bool cluster_ok) {
+// Blocks a plan launches per launch.
+int plan_blocks(const Plan& pl) {
+  return pl.nseg > 1 ? pl.n_chains * pl.nseg : (pl.n_chains + pl.chains_per_block - 1) / pl.chains_per_block;
+}
+
+// `nsm`: streaming multiprocessors of the device the plan is for (148 on a B200).
+CallPlan plan_call(const Shape& s, bool tma, bool cluster_ok, int nsm) {
   CallPlan cp{};
   cp.tma = tma;
   const int ng = states_per_lane(s.N);
@@ -301,6 +307,10 @@ CallPlan plan_call(const Shape& s, bool tma, bool cluster_ok) {
   }
   if (!cp.smem_multi) {
     cp.pl = make_plan(s, ng, ng >= 16, tma);
+    // two channels per lane share the B, C loads, but halve the number of chains: when that
+    // leaves most multiprocessors idle (few channels, e.g. batch 1 with a small map), one
+    // channel per lane and twice the chains is faster
+    if (plan_blocks(cp.pl) * 2 <= nsm) cp.pl = make_plan(s, ng, true, tma);
     cp.yacc_stride = 0;
     cp.smem = cp.pl.carry_smem + cp.pl.tile_smem;
   }
@@ -314,8 +324,7 @@ CallPlan plan_call(const Shape& s, bool tma, bool cluster_ok) {
   cp.yacc_bytes = cp.need_yacc_ws ? s.xy_count * sizeof(float) : 0;
   cp.need_ws = cp.link == kLinkGlobal || cp.need_yacc_ws;
   cp.ws_bytes = cp.need_ws ? sync_bytes(cp.link == kLinkGlobal ? cp.items : 0) + cp.carry_bytes + cp.yacc_bytes : 0;
-  cp.grid = pl.nseg > 1 ? pl.n_chains * pl.nseg
-                        : (pl.n_chains + pl.chains_per_block - 1) / pl.chains_per_block;
+  cp.grid = plan_blocks(pl);
   cp.launches = cp.global_multi ? cp.nk : 1;
   return cp;
 }
@@ -423,7 +432,7 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
   TmaMaps tm;
   std::memset(&tm, 0, sizeof tm);
   bool tma = tma_possible(s, x, delta, B, C);
-  CallPlan cp = plan_call(s, tma, true);
+  CallPlan cp = plan_call(s, tma, true, nsm);
   if (tma) {
     const Plan& p0 = cp.pl;
     const int nb = kQ * p0.var.ng;
@@ -431,13 +440,13 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
           encode_map(&tm.d, delta, s.bf16, W, H, channels, batch, p0.var.cmax, p0.cpw) &&
           encode_map(&tm.b, B, s.bf16, W, H, N, static_cast<long long>(batch) * s.K, p0.var.cmax, nb) &&
           encode_map(&tm.c, C, s.bf16, W, H, N, static_cast<long long>(batch) * s.K, p0.var.cmax, nb);
-    if (!tma) cp = plan_call(s, false, true);
+    if (!tma) cp = plan_call(s, false, true, nsm);
   }
   // a chain's blocks share distributed shared memory when such a cluster fits on the device
   if (cp.link == kLinkCluster &&
       !cluster_worth_it(tma ? cp.pl.var.fn_tma : cp.pl.var.fn_plain, cp.pl.warps * 32, cp.smem, cp.pl.nseg,
                         cp.pl.n_chains))
-    cp = plan_call(s, tma, false);
+    cp = plan_call(s, tma, false, nsm);
   const Plan& pl = cp.pl;
   const KernelFn fn = tma ? pl.var.fn_tma : pl.var.fn_plain;
 
@@ -589,7 +598,7 @@ int scan2d_query_plan(int batch, int channels, int H, int W, int N, unsigned fla
   const bool tma = (static_cast<size_t>(W) * s.in_elem) % 16 == 0;
   // chains of up to 16 blocks are planned as clusters (the call itself falls back to the
   // global ring if such a cluster cannot be resident on the device)
-  const scan2d::CallPlan cp = scan2d::plan_call(s, tma, true);
+  const scan2d::CallPlan cp = scan2d::plan_call(s, tma, true, 148);   // planned for a B200
   const long long v[SCAN2D_PLAN_FIELDS] = {
       cp.launches, cp.grid, cp.pl.warps * 32, static_cast<long long>(cp.smem), cp.pl.nseg,
       cp.pl.var.cmax, cp.pl.wpc, cp.smem_multi ? 1 : (cp.global_multi ? 2 : 0), cp.pl.var.ng,

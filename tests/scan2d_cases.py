@@ -33,6 +33,9 @@ CASES = {
     "random_A": ("giga", dict(channels=8, H=48, W=100, random_A=True)),
     "wsi_mask_recipe": ("wsi", dict(channels=16, H=40, W=56)),
     "giga_recipe_small": ("giga", dict(channels=8, H=64, W=300)),
+    # enough channel groups that the planner keeps two channels per lane
+    "f32_g2_chain_tma": ("tiny", dict(batch=4, channels=160, N=16, H=6, W=128)),
+    "bf16_g2_14x14": ("small", dict(batch=64, channels=80, H=10, W=14)),
 }
 for n in (1, 3, 5, 8, 12, 17, 32, 33, 64):
     CASES[f"N{n}"] = ("tiny", dict(batch=1, channels=9, N=n, H=9, W=23))
