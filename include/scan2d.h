@@ -91,6 +91,9 @@ extern "C" {
  *   flags             : SCAN2D_BF16 | SCAN2D_OUT_F32 | orientation bits;
  *   stream            : a cudaStream_t (NULL = the legacy default stream).
  * Asynchronous: returns once the work is enqueued on `stream`.  y must not alias an input.
+ * Repeated calls give bitwise identical y, except that when several orientations are summed
+ * in shared memory (small maps) the order of those fp32 additions depends on timing, so y
+ * may differ in the last bits.
  * Returns 0, or SCAN2D_E_NULL / _DIMS / _N / _FLAGS / _ALIGN / _NOMEM / _LAUNCH / _DEVICE.
  */
 int scan2d_fwd(const void *x, const void *delta, const float *A, const void *B, const void *C,
@@ -109,8 +112,7 @@ int scan2d_fwd(const void *x, const void *delta, const float *A, const void *B, 
  * accumulator of several orientations with bf16 output on maps too large for shared memory)
  * from one fixed device array of SCAN2D_NOALLOC_SCRATCH_BYTES that the library holds on every
  * device that loads it, until the process exits.  It calls no cudaMalloc, cudaFree or other
- * allocating routine.  Arguments, layouts and results are those of scan2d_fwd (y is
- * bitwise the same for the same launch plan).
+ * allocating routine.  Arguments, layouts and results are those of scan2d_fwd.
  *   - The first call on a device looks up the array's device address with that device
  *     current; make that first call before any stream capture.
  *   - Every call, on every stream, shares the one array and leaves its contents behind; each

@@ -20,6 +20,7 @@ namespace {
 constexpr long long kTimeoutNs = 2000000000LL;   // bounded inter-block waits: 2 s
 constexpr size_t kAlign = 256;
 constexpr size_t kSmemBudget = 200 * 1024;       // dynamic shared memory per block we plan for
+constexpr size_t kSmemBudgetSplit = 220 * 1024;  // ... for blocks whose chains split the orientations
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -70,15 +71,21 @@ struct Variant {
   size_t tile_bytes_plain;    // one staged strip row (plain-load path)
   size_t carry_slot_bytes;    // one carry row of a warp
   KernelFn fn_tma, fn_plain;
+  KernelFn fn_tma16, fn_plain16;   // up to 16 warps per block (one channel per lane only)
 };
 
 template <typename Tin, int NG, int G, int CMAX>
 Variant make_variant() {
   using LT = Layout<Tin, NG, G, CMAX, kTileRows>;
   using LP = Layout<Tin, NG, G, CMAX, 1>;
-  return Variant{NG, G, CMAX, static_cast<size_t>(LT::TILE_BYTES), static_cast<size_t>(LP::TILE_BYTES),
-                 static_cast<size_t>(LP::CARRY_SLOT_BYTES),
-                 scan2d_kernel<Tin, NG, G, CMAX, true>, scan2d_kernel<Tin, NG, G, CMAX, false>};
+  Variant v{NG, G, CMAX, static_cast<size_t>(LT::TILE_BYTES), static_cast<size_t>(LP::TILE_BYTES),
+            static_cast<size_t>(LP::CARRY_SLOT_BYTES),
+            scan2d_kernel<Tin, NG, G, CMAX, true>, scan2d_kernel<Tin, NG, G, CMAX, false>, nullptr, nullptr};
+  if constexpr (G == 1) {
+    v.fn_tma16 = scan2d_kernel<Tin, NG, G, CMAX, true, kMaxWarpsSplit>;
+    v.fn_plain16 = scan2d_kernel<Tin, NG, G, CMAX, false, kMaxWarpsSplit>;
+  }
+  return v;
 }
 
 int states_per_lane(int N) {
@@ -263,6 +270,7 @@ struct CallPlan {
   int codes[4], nk;
   bool smem_multi, global_multi, need_yacc_ws, need_ws;
   int link, yacc_stride, grid, launches;
+  int orient_split;            // 2: two chain slots per block walk every other orientation
   size_t smem, items, carry_bytes, yacc_bytes, ws_bytes;
 };
 
@@ -275,6 +283,7 @@ int plan_blocks(const Plan& pl) {
 CallPlan plan_call(const Shape& s, bool tma, bool cluster_ok, int nsm) {
   CallPlan cp{};
   cp.tma = tma;
+  cp.orient_split = 1;
   const int ng = states_per_lane(s.N);
   cp.nk = 0;
   for (int o = 0; o < 4; ++o)
@@ -293,7 +302,22 @@ CallPlan plan_call(const Shape& s, bool tma, bool cluster_ok, int nsm) {
                                (p1.tile_smem + p1.carry_smem) / p1.chains_per_block;
       int cpb = p1.chains_per_block;
       while (cpb > 1 && per_chain * cpb > kSmemBudget) --cpb;
-      if (per_chain * cpb <= kSmemBudget) {
+      // one chain per block: let a second chain slot walk every other orientation of the same
+      // channels at the same time (twice the warps, half the walk), if that still fits
+      const size_t split_smem = sizeof(float) * p1.cpw * stride + 2 * (p1.tile_smem + p1.carry_smem);
+      // (up to 4 states per lane: the 16-warp variants get 128 registers a thread)
+      if (p1.chains_per_block == 1 && 2 * p1.wpc <= kMaxWarpsSplit && split_smem <= kSmemBudgetSplit &&
+          p1.var.fn_tma16 != nullptr && ng <= 4) {
+        p1.tile_smem *= 2;
+        p1.carry_smem *= 2;
+        p1.chains_per_block = 2;
+        p1.warps = 2 * p1.wpc;
+        cp.pl = p1;
+        cp.smem_multi = true;
+        cp.orient_split = 2;
+        cp.yacc_stride = stride;
+        cp.smem = split_smem;
+      } else if (per_chain * cpb <= kSmemBudget) {
         p1.tile_smem = p1.tile_smem / p1.chains_per_block * cpb;
         p1.carry_smem = p1.carry_smem / p1.chains_per_block * cpb;
         p1.chains_per_block = cpb;
@@ -324,7 +348,7 @@ CallPlan plan_call(const Shape& s, bool tma, bool cluster_ok, int nsm) {
   cp.yacc_bytes = cp.need_yacc_ws ? s.xy_count * sizeof(float) : 0;
   cp.need_ws = cp.link == kLinkGlobal || cp.need_yacc_ws;
   cp.ws_bytes = cp.need_ws ? sync_bytes(cp.link == kLinkGlobal ? cp.items : 0) + cp.carry_bytes + cp.yacc_bytes : 0;
-  cp.grid = plan_blocks(pl);
+  cp.grid = cp.orient_split > 1 ? pl.n_chains : plan_blocks(pl);
   cp.launches = cp.global_multi ? cp.nk : 1;
   return cp;
 }
@@ -448,7 +472,8 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
                         cp.pl.n_chains))
     cp = plan_call(s, tma, false, nsm);
   const Plan& pl = cp.pl;
-  const KernelFn fn = tma ? pl.var.fn_tma : pl.var.fn_plain;
+  const KernelFn fn = cp.orient_split > 1 ? (tma ? pl.var.fn_tma16 : pl.var.fn_plain16)
+                                         : (tma ? pl.var.fn_tma : pl.var.fn_plain);
 
   Params prm;
   std::memset(&prm, 0, sizeof prm);
@@ -460,6 +485,7 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
   prm.link = cp.link;
   prm.timeout_ns = kTimeoutNs;
   prm.yacc_stride = cp.yacc_stride;
+  prm.orient_split = cp.orient_split;
   prm.out_f32 = s.out_f32 ? 1 : 0;
   prm.vec_store = (W % 4 == 0) && aligned(y, s.out_f32 ? 16 : 8);
 

@@ -53,7 +53,8 @@ constexpr int kQ = 4;                  // state-group lanes per channel group
 constexpr int kGroups = 8;             // channel groups per warp
 constexpr int kRing = 16;              // carry rows buffered in global memory between blocks
 constexpr int kCarryRing = 4;          // carry rows buffered in shared memory between warps
-constexpr int kMaxWarps = 8;           // compute warps per block (plus one TMA producer warp)
+constexpr int kMaxWarps = 8;           // warps per block, except for split orientations
+constexpr int kMaxWarpsSplit = 16;     // warps per block when two chains split the orientations
 constexpr int kTileRows = 4;           // rows per staged tile (TMA path; the plain path stages 1)
 constexpr int kTileDepth = 2;          // staged tiles in flight per warp (TMA path)
 constexpr int kPublish = 4;            // global fallback: rows per flag release
@@ -95,6 +96,8 @@ struct Params {
   int orient_k[4];          // index of the orientation's B_k, C_k
   int mode;
   int yacc_stride;          // kSmemMulti: floats per channel in shared memory
+  int orient_split;         // kSmemMulti: 2 when the block's two chain slots walk every other
+                            // orientation of the same channels (else 1)
   int vec_store;            // rows of y are aligned for 4-column vector stores
   int out_f32;              // y is fp32 (else bf16)
   unsigned long long* ctrl;   // [0] ticket counter, [1] finished blocks, [2] aborted generation
@@ -385,8 +388,8 @@ __host__ __device__ constexpr size_t carry_ring_bytes(int warps) {
 }
 
 // ---- the kernel ------------------------------------------------------------------------------
-template <typename Tin, int NG, int G, int CMAX, bool TMA>
-__global__ void __launch_bounds__(kMaxWarps * 32, 1)
+template <typename Tin, int NG, int G, int CMAX, bool TMA, int MAXW = kMaxWarps>
+__global__ void __launch_bounds__(MAXW * 32, 1)
 scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps tm) {
   constexpr int R = TMA ? kTileRows : 1;                     // rows per staged tile
   using L = Layout<Tin, NG, G, CMAX, R>;
@@ -400,9 +403,9 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   constexpr int NP = L::NP;
 
   extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ uint64_t s_tfull[kMaxWarps][kTileDepth];        // staged tile landed (TMA)
-  __shared__ uint64_t s_full[kMaxWarps][kCarryRing];         // carry slot written (consumer side)
-  __shared__ uint64_t s_empty[kMaxWarps][kCarryRing];        // carry slot read (producer side)
+  __shared__ uint64_t s_tfull[MAXW][kTileDepth];             // staged tile landed (TMA)
+  __shared__ uint64_t s_full[MAXW][kCarryRing];              // carry slot written (consumer side)
+  __shared__ uint64_t s_empty[MAXW][kCarryRing];             // carry slot read (producer side)
   __shared__ int s_item;
 
   const unsigned FULL = 0xffffffffu;
@@ -428,6 +431,7 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   auto chain_of = [&](int sl) -> int {
     if (cluster) return blockIdx.x / p.nseg;
     if (global_link) return s_item / p.nseg;
+    if (p.orient_split > 1) return blockIdx.x;               // the slots share the channels
     return blockIdx.x * p.chains_per_block + sl;
   };
   const int chain = chain_of(slot);
@@ -469,6 +473,12 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   unsigned char* tiles0 = smem + carry_ring_bytes<Tin, NG, G, CMAX>(ncomp);
   unsigned char* tiles = tiles0 + (is_compute ? warp : 0) * DEPTH * L::TILE_BYTES;
   float* yacc_s = reinterpret_cast<float*>(tiles0 + static_cast<size_t>(ncomp) * DEPTH * L::TILE_BYTES);
+  const int yslot = p.orient_split > 1 ? 0 : slot;           // accumulator of this warp's chain
+  if (p.mode == kSmemMulti) {
+    // the orientations add into the accumulator (in any order, from any warp): start at zero
+    const int ny = (p.orient_split > 1 ? 1 : p.chains_per_block) * L::CPW * p.yacc_stride;
+    for (int e = threadIdx.x; e < ny; e += blockDim.x) yacc_s[e] = 0.f;
+  }
   auto carry_slot = [&](int wr, int s) -> float* {
     return reinterpret_cast<float*>(carry_base + (wr * kCarryRing + s) * L::CARRY_SLOT_BYTES);
   };
@@ -493,12 +503,17 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   else __syncthreads();
 
   const int item = chain * p.nseg + seg;
-  const int U = p.orient_count * H;                          // rows each warp walks
+  // orientations this warp walks: all of them, or every other one when two chains split them
+  const int ostep = p.orient_split > 1 ? p.orient_split : 1;
+  const int oi_first = ostep > 1 ? slot : 0;
+  const int n_or = oi_first < p.orient_count ? (p.orient_count - oi_first + ostep - 1) / ostep : 0;
+  const int U = n_or * H;                                    // rows each warp walks
 
   // row uu of the walk of the warp at scan position us -> (orientation, stored row, stored strip)
   auto row_coords_of = [&](int us, int uu, int& oi, int& i, int& t) {
-    oi = uu / H;
-    const int r = uu - oi * H;
+    const int oj = uu / H;
+    const int r = uu - oj * H;
+    oi = oi_first + oj * ostep;
     const int o = p.orient_code[oi];
     i = (o & 2) ? H - 1 - r : r;
     t = (o & 1) ? p.strips - 1 - us : us;
@@ -560,11 +575,11 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   // a slot right after all its lanes have read the tile's last row.  Once a wait of this warp
   // has given up, nothing more is staged.
   const int TPO = (H + R - 1) / R;                           // tiles per orientation
-  const int UT = p.orient_count * TPO;                       // tiles of the walk
+  const int UT = n_or * TPO;                                 // tiles of the walk
   int staged = 0;                                            // tiles of the walk staged so far
   // the next tile to stage, as (orientation, tile in it), with that orientation's stored strip
   // column, flip and B/C index (lane 0's copy is the one in use)
-  int st_oi = 0, st_tr = 0, st_col = 0, st_flip = 0, st_bk = 0;
+  int st_oi = oi_first, st_tr = 0, st_col = 0, st_flip = 0, st_bk = 0;
   auto st_orientation = [&]() {
     const int o = p.orient_code[st_oi];
     st_flip = o & 2;
@@ -583,7 +598,7 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
     tma_load_4d(dst + L::C_OFF * L::ESZ, &tm.c, bar, st_col, 0, row0, st_bk);
     if (++st_tr == TPO) {
       st_tr = 0;
-      if (++st_oi < p.orient_count) st_orientation();
+      if ((st_oi += ostep) < p.orient_count) st_orientation();
     }
   };
   if (TMA && strip_ok) {
@@ -641,7 +656,8 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
 
   unsigned long long ack_seen = 0;                           // global ring: last ack read
   int u = 0;                                                 // rows of the walk done so far
-  for (int oi = 0; oi < p.orient_count; ++oi) {
+  for (int oj = 0; oj < n_or; ++oj) {
+    const int oi = oi_first + oj * ostep;
     const int o = p.orient_code[oi];
     const bool flipW = (o & 1) != 0, flipH = (o & 2) != 0;
     const int t = flipW ? p.strips - 1 - u_scan : u_scan;   // stored strip
@@ -717,10 +733,10 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
             if (gc + m < W) store_out(p.y, rowoff + gc + m, own[m], p.out_f32);
         }
       } else if (p.mode == kSmemMulti) {
-        float* a = yacc_s + (slot * L::CPW + cg * G + c) * p.yacc_stride + i_row * W + gc;
+        float* a = yacc_s + (yslot * L::CPW + cg * G + c) * p.yacc_stride + i_row * W + gc;
 #pragma unroll
         for (int m = 0; m < E / 4; ++m)
-          if (gc + m < W) a[m] = (oi == 0) ? own[m] : a[m] + own[m];
+          if (gc + m < W) atomicAdd(a + m, own[m]);
       } else {
 #pragma unroll
         for (int m = 0; m < E / 4; ++m) {
@@ -736,7 +752,7 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
     for (int r = 0; r < H && strip_ok; ++r, ++u) {
       const int i = flipH ? H - 1 - r : r;
       const int tr = r / R, rr = r - tr * R;                 // tile of the orientation, row in it
-      const int wt = oi * TPO + tr;                          // tile of the walk
+      const int wt = oj * TPO + tr;                          // tile of the walk
       const int s = wt % DEPTH;
       const int rt = flipH ? R - 1 - rr : rr;                // this row's place in the staged tile
       const Tin* tile = reinterpret_cast<const Tin*>(tiles + s * L::TILE_BYTES);
@@ -932,10 +948,6 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
       reduce_row(pacc, own_last);
       write_row(p_i, own_last);
     }
-    // orientations summed in shared memory: no compute warp may start the next orientation
-    // (whose strips map to other columns) before every compute warp has finished this one
-    if (p.mode == kSmemMulti && is_compute)
-      asm volatile("bar.sync 1, %0;" ::"r"(ncomp * 32) : "memory");
   }
   // ---- after a timed-out wait: let this warp's copies still in flight land (bounded) -------
   if (TMA && aborted && lane == 0) {
@@ -948,12 +960,13 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
 
   // ---- kSmemMulti: write the accumulated maps of this block's chains --------------------------
   if (p.mode == kSmemMulti && chain_ok) {
-    const int nthreads = p.wpc * 32;
-    const int tid = w * 32 + lane;
+    // every warp of the chain (both slots when they split the orientations) writes a share
+    const int nthreads = (p.orient_split > 1 ? ncomp : p.wpc) * 32;
+    const int tid = (p.orient_split > 1 ? warp : w) * 32 + lane;
     for (int cs = 0; cs < L::CPW; ++cs) {
       const int dd = grp * L::CPW + cs;
       if (dd >= p.channels) break;
-      const float* src = yacc_s + (slot * L::CPW + cs) * p.yacc_stride;
+      const float* src = yacc_s + (yslot * L::CPW + cs) * p.yacc_stride;
       const size_t base = (static_cast<size_t>(b) * p.channels + dd) * HW;
       for (size_t e = tid; e < HW; e += nthreads) store_out(p.y, base + e, src[e], p.out_f32);
     }

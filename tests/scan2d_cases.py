@@ -36,6 +36,10 @@ CASES = {
     # enough channel groups that the planner keeps two channels per lane
     "f32_g2_chain_tma": ("tiny", dict(batch=4, channels=160, N=16, H=6, W=128)),
     "bf16_g2_14x14": ("small", dict(batch=64, channels=80, H=10, W=14)),
+    # two chain slots per block, each walking every other orientation
+    "bf16_k4_split_plain": ("vision", dict(batch=1, channels=8, H=9, W=44)),
+    "bf16_k3_split_plain": ("vision", dict(batch=2, channels=8, H=11, W=41, orient_mask=0b0111)),
+    "f32_k2_split_tma": ("tiny", dict(batch=1, channels=8, N=16, H=12, W=48, orient_mask=0b0011)),
 }
 for n in (1, 3, 5, 8, 12, 17, 32, 33, 64):
     CASES[f"N{n}"] = ("tiny", dict(batch=1, channels=9, N=n, H=9, W=23))

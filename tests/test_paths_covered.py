@@ -36,6 +36,9 @@ def test_every_path_is_exercised(plans):
     assert any(p["link"] == 2 and p["tma"] == 1 for p in ps), "global-ring chain, TMA"
     assert any(p["link"] == 2 and p["tma"] == 0 for p in ps), "global-ring chain, plain"
     assert any(p["link"] == 1 and p["nseg"] == 16 for p in ps), "the largest cluster"
+    split = [p for p in ps if p["mode"] == 1 and p["threads"] > 256]
+    assert any(p["tma"] == 1 for p in split) and any(p["tma"] == 0 for p in split), \
+        "two chain slots splitting the orientations, TMA and plain staging"
 
 
 def test_long_chain_hits_ring_back_pressure(plans):
