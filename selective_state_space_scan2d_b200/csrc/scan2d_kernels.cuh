@@ -259,14 +259,14 @@ __device__ __noinline__ void report_timeout(unsigned long long* ctrl, unsigned l
 __device__ __noinline__ bool wait_geq(const unsigned long long* p, unsigned long long want,
                                       unsigned long long* ctrl, unsigned long long gen,
                                       long long timeout_ns) {
-  long long t0 = 0;
-  for (unsigned it = 0;; ++it) {
+  long long t0 = -1;
+  for (unsigned it = 1;; ++it) {
     if (ld_acquire(p) >= want) return true;
     if ((it & 31u) == 0u) {
       if (ld_acquire(&ctrl[2]) == gen) return false;
       const long long now = global_ns();
-      if (it == 0u) t0 = now;
-      if (now - t0 > timeout_ns || it > (1u << 30)) {
+      if (t0 < 0) t0 = now;
+      else if (now - t0 > timeout_ns || it > (1u << 30)) {
         report_timeout(ctrl, gen);
         return false;
       }
@@ -279,11 +279,14 @@ __device__ __noinline__ bool wait_geq(const unsigned long long* p, unsigned long
 // time runs out.  Returns false after a time-out (the error is recorded).
 __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, unsigned parity, unsigned long long* ctrl,
                                             unsigned long long gen, long long timeout_ns) {
-  const long long t0 = global_ns();
+  // the clock is read only every 64 tries (most waits end well before the first read)
+  long long t0 = -1;
   for (unsigned it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 15u) == 0u) {
-      if (global_ns() - t0 > timeout_ns || it > (1u << 28)) {
+    if ((it & 63u) == 0u) {
+      const long long now = global_ns();
+      if (t0 < 0) t0 = now;
+      else if (now - t0 > timeout_ns || it > (1u << 28)) {
         report_timeout(ctrl, gen);
         return false;
       }
@@ -639,13 +642,15 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   // reloads row uu until every tag is right; true if it gave up (time-out or aborted launch)
   auto cw_poll = [&](int uu) -> bool {
     const unsigned want = ctag(p.gen, uu);
-    const long long t0 = global_ns();
+    long long t0 = -1;
     for (unsigned it = 1;; ++it) {
       if (cw_ready(want)) return false;
       __nanosleep(32);
       if ((it & 15u) == 0u) {
         if (ld_acquire(&p.ctrl[2]) == p.gen) return true;
-        if (global_ns() - t0 > p.timeout_ns || it > (1u << 26)) {
+        const long long now = global_ns();
+        if (t0 < 0) t0 = now;
+        else if (now - t0 > p.timeout_ns || it > (1u << 26)) {
           report_timeout(p.ctrl, p.gen);
           return true;
         }
