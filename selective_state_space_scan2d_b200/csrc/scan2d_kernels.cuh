@@ -248,6 +248,27 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// The four copies of one staged tile (x, delta, B, C boxes) and the arming of their mbarrier,
+// issued by one lane chosen with elect.sync.  Called by every lane of a converged warp, so the
+// operands are warp-uniform and no lane waits in a divergent branch.
+__device__ __forceinline__ void tma_tile4(uint32_t bar, uint32_t dx, uint32_t dd, uint32_t db, uint32_t dc,
+                                          const CUtensorMap* mx, const CUtensorMap* md, const CUtensorMap* mb,
+                                          const CUtensorMap* mc, int col, int ch, int row, int bx, int bk,
+                                          unsigned tx_bytes) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "@p mbarrier.arrive.expect_tx.relaxed.cta.shared::cta.b64 _, [%0], %14;\n\t"
+      "@p cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%1], [%5, {%9, %10, %11, %12}], [%0];\n\t"
+      "@p cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%2], [%6, {%9, %10, %11, %12}], [%0];\n\t"
+      "@p cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%3], [%7, {%9, %15, %11, %13}], [%0];\n\t"
+      "@p cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%4], [%8, {%9, %15, %11, %13}], [%0];\n\t"
+      "}" ::"r"(bar), "r"(dx), "r"(dd), "r"(db), "r"(dc),
+      "l"(reinterpret_cast<uint64_t>(mx)), "l"(reinterpret_cast<uint64_t>(md)), "l"(reinterpret_cast<uint64_t>(mb)),
+      "l"(reinterpret_cast<uint64_t>(mc)), "r"(col), "r"(ch), "r"(row), "r"(bx), "r"(bk), "r"(tx_bytes), "r"(0)
+      : "memory");
+}
+
 // Records a device error once and marks this launch generation aborted: every other wait of
 // the launch then gives up at once (checked through ctrl[2] where a ctrl block exists).
 __device__ __noinline__ void report_timeout(unsigned long long* ctrl, unsigned long long gen) {
@@ -589,16 +610,13 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
     st_col = ((o & 1) ? p.strips - 1 - u_scan : u_scan) * CMAX;
     st_bk = b * p.K + p.orient_k[st_oi];
   };
-  auto stage_tile = [&]() {                                  // lane 0 only: walk tile `staged`
+  auto stage_tile = [&]() {                                  // whole warp, converged: walk tile `staged`
     const int row0 = st_flip ? H - R - st_tr * R : st_tr * R;  // first stored row of the box
     const int s = staged % DEPTH;
-    unsigned char* dst = tiles + s * L::TILE_BYTES;
-    uint64_t* bar = &s_tfull[warp][s];
-    mbar_arm_tx(smem_u32(bar), L::TX_BYTES);
-    tma_load_4d(dst + L::X_OFF * L::ESZ, &tm.x, bar, st_col, grp * L::CPW, row0, b);
-    tma_load_4d(dst + L::D_OFF * L::ESZ, &tm.d, bar, st_col, grp * L::CPW, row0, b);
-    tma_load_4d(dst + L::B_OFF * L::ESZ, &tm.b, bar, st_col, 0, row0, st_bk);
-    tma_load_4d(dst + L::C_OFF * L::ESZ, &tm.c, bar, st_col, 0, row0, st_bk);
+    const uint32_t dst = smem_u32(tiles + s * L::TILE_BYTES);
+    tma_tile4(smem_u32(&s_tfull[warp][s]), dst + L::X_OFF * L::ESZ, dst + L::D_OFF * L::ESZ,
+              dst + L::B_OFF * L::ESZ, dst + L::C_OFF * L::ESZ, &tm.x, &tm.d, &tm.b, &tm.c, st_col,
+              grp * L::CPW, row0, b, st_bk, L::TX_BYTES);
     if (++st_tr == TPO) {
       st_tr = 0;
       if ((st_oi += ostep) < p.orient_count) st_orientation();
@@ -606,11 +624,8 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   };
   if (TMA && strip_ok) {
     const int first = UT < DEPTH ? UT : DEPTH;
-    if (lane == 0) {
-      st_orientation();
-      for (; staged < first; ++staged) stage_tile();
-    }
-    staged = first;
+    st_orientation();
+    for (; staged < first; ++staged) stage_tile();
   }
 
   // where this warp's carries go: the next warp of this block, or warp 0 of the next block
@@ -926,10 +941,13 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
       }
 
       // ---- (5) refill the tile slot (every lane has read the tile's last row) ---------------
+      // a wait that gave up on one lane gives up for the warp: the refill below is issued by
+      // the converged warp
       __syncwarp();
+      aborted = __any_sync(FULL, aborted);
       if (TMA && (rr == R - 1 || r == H - 1) && !aborted && staged < UT) {
         // every lane has read the tile's last row (its values are in use): refill the slot
-        if (lane == 0) stage_tile();
+        stage_tile();
         ++staged;
       }
       // a carry slot filled by the previous block: re-arm it for its next use, then free it;
