@@ -439,7 +439,13 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   const int ncomp = p.wpc * p.chains_per_block;
   const bool is_compute = warp < ncomp;
   const int slot = is_compute ? warp / p.wpc : 0;            // chain slot inside the block
-  const int w = is_compute ? warp - slot * p.wpc : 0;        // strip inside the segment
+  // Warp k runs on sub-partition k % 4 of the SM.  With one chain of 8 strips per block, the
+  // two warps of a sub-partition take adjacent strips (strip s on warp s/2 + 4 (s % 2)): a warp
+  // then computes while its partner waits for the carry it is about to hand over, instead of
+  // both computing (or both waiting) at the same time.
+  const bool pair_map = p.wpc == 8 && p.chains_per_block == 1;
+  auto warp_of = [&](int ws) { return pair_map ? (ws >> 1) + 4 * (ws & 1) : slot * p.wpc + ws; };
+  const int w = is_compute ? (pair_map ? 2 * (warp & 3) + (warp >> 2) : warp - slot * p.wpc) : 0;  // strip
   const int cg = lane >> 2;                 // channel group
   const int q = lane & 3;                   // state group
   const bool cluster = p.link == kLinkCluster;
@@ -629,7 +635,7 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   }
 
   // where this warp's carries go: the next warp of this block, or warp 0 of the next block
-  const uint32_t next_full0 = smem_u32(&s_full[next_local ? warp + 1 : 0][0]);
+  const uint32_t next_full0 = smem_u32(&s_full[next_local ? warp_of(w + 1) : 0][0]);
   const uint32_t my_empty0 = smem_u32(&s_empty[warp][0]);
   uint32_t next_ring_cl = 0, next_full_cl = 0, prev_empty_cl = 0;
   if (cluster) {
@@ -637,7 +643,7 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
       next_ring_cl = map_rank(smem_u32(carry_slot(0, 0)), seg + 1);
       next_full_cl = map_rank(smem_u32(&s_full[0][0]), seg + 1);
     }
-    if (left_remote) prev_empty_cl = map_rank(smem_u32(&s_empty[p.wpc - 1][0]), seg - 1);
+    if (left_remote) prev_empty_cl = map_rank(smem_u32(&s_empty[warp_of(p.wpc - 1)][0]), seg - 1);
   }
 
   // global ring, consumer side: this lane's tagged words of the row it will need next
@@ -819,7 +825,7 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
 #pragma unroll
           for (int g = 0; g < NG; ++g) hh[c][g] = in[c * NG + g];
         // free the slot (a slot filled from another block is freed once its values are used)
-        if (!left_remote) mbar_arrive_local(smem_u32(&s_empty[warp - 1][cs]));
+        if (!left_remote) mbar_arrive_local(smem_u32(&s_empty[warp_of(w - 1)][cs]));
       } else {
 #pragma unroll
         for (int c = 0; c < G; ++c)
@@ -897,7 +903,7 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
 #pragma unroll
           for (int g = 0; g < NG; ++g) out[c * NG + g] = hh[c][g];
         if (next_local) {
-          float4* dst = reinterpret_cast<float4*>(carry_slot(warp + 1, cs)) + lane * (L::CARRY_PAD / 4);
+          float4* dst = reinterpret_cast<float4*>(carry_slot(warp_of(w + 1), cs)) + lane * (L::CARRY_PAD / 4);
 #pragma unroll
           for (int k4 = 0; k4 < L::CARRY_PAD / 4; ++k4)
             dst[k4] = make_float4(out[4 * k4], out[4 * k4 + 1], out[4 * k4 + 2], out[4 * k4 + 3]);
