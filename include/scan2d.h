@@ -16,6 +16,13 @@
  * states, the skip term and the orientation semantics are not printed on the pages; the
  * plainest readings are taken (see the design notes shipped with the repository).
  *
+ * Scan order (papernotes.org notes, "消融实验要点": horizontal-then-vertical and
+ * vertical-then-horizontal are both studied).  With SCAN2D_VFIRST the two recurrences run in
+ * the other order, with the same Abar, Bbar, C and zero initial states:
+ *     vv[i,j] = Abar[i,j] * vv[i-1,j] + Bbar[i,j] * x[i,j]      (vertical first)
+ *     h[i,j]  = Abar[i,j] * h[i,j-1]  + vv[i,j]                 (then horizontal)
+ * which equals the default order on the transposed map, transposed back.
+ *
  * Orientations ("reverse scans" in the papernotes "局限与展望", "四象限" in the juejin
  * section 七.4): orientation TL scans from the top-left corner; TR from the top-right
  * (W reversed); BL from the bottom-left (H reversed); BR from the bottom-right.  Each
@@ -57,12 +64,13 @@ extern "C" {
 /* ---- flags ----------------------------------------------------------------------- */
 #define SCAN2D_BF16     0x1u   /* x, delta, B, C (and y) are bf16 instead of fp32      */
 #define SCAN2D_OUT_F32  0x2u   /* with SCAN2D_BF16: y is fp32                          */
+#define SCAN2D_VFIRST   0x8u   /* scan order: vertical scan first, then horizontal      */
 #define SCAN2D_OR_TL    0x10u  /* orientation: from the top-left corner (default)     */
 #define SCAN2D_OR_TR    0x20u  /* from the top-right corner (W reversed)              */
 #define SCAN2D_OR_BL    0x40u  /* from the bottom-left corner (H reversed)            */
 #define SCAN2D_OR_BR    0x80u  /* from the bottom-right corner (H and W reversed)     */
 #define SCAN2D_OR_ALL   0xF0u
-#define SCAN2D_FLAGS_KNOWN 0xF3u
+#define SCAN2D_FLAGS_KNOWN 0xFBu
 
 /* ---- limits ---------------------------------------------------------------------- */
 #define SCAN2D_MAX_N    64     /* states per channel                                   */
@@ -88,7 +96,7 @@ extern "C" {
  *   x, delta, B, C, y : device pointers, element type per flags (see above);
  *   A, Dskip          : device pointers to fp32 (Dskip may be NULL);
  *   batch, channels, H, W >= 1;  1 <= N <= SCAN2D_MAX_N;
- *   flags             : SCAN2D_BF16 | SCAN2D_OUT_F32 | orientation bits;
+ *   flags             : SCAN2D_BF16 | SCAN2D_OUT_F32 | SCAN2D_VFIRST | orientation bits;
  *   stream            : a cudaStream_t (NULL = the legacy default stream).
  * Asynchronous: returns once the work is enqueued on `stream`.  y must not alias an input.
  * Repeated calls give bitwise identical y, except that when several orientations are summed

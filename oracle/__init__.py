@@ -14,7 +14,8 @@ Input conventions (numpy):
     bf16 bit patterns (numpy has no bf16 dtype).  Every stored value is widened exactly.
   * x, delta: (batch, channels, H, W); A: (channels, N) float32; B, C: (batch, K, N, H, W);
     Dskip: (channels,) float32 or None.
-  * ``orient_mask``: bit 0 top-left, bit 1 top-right (flip W), bit 2 bottom-left (flip H),
+  * ``orient_mask``: bit 4 (0x10) selects the vertical-then-horizontal scan order.
+  * ``orient_mask`` bits 0-3: bit 0 top-left, bit 1 top-right (flip W), bit 2 bottom-left (flip H),
     bit 3 bottom-right (flip both).  K = number of set bits.
 """
 from __future__ import annotations

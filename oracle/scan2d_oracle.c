@@ -25,6 +25,13 @@
  * The same Abar is used in both scans and the vertical scan adds no second Bbar
  * ([J 4.5(2)] writes Abar_{i,j} and h^hor_{i,j} only).
  *
+ * Scan order ([PN 消融实验要点]: horizontal-then-vertical and vertical-then-horizontal are
+ * both studied; READING: the same two recurrences in the other order).  With bit 4 of the
+ * mask set, each (b, d, n) map is scanned vertical-first:
+ *   vv[i,j]    = Abar[i,j]*vv[i-1,j] + Bbar[i,j]*x[i,j]          vv[-1,j] = 0
+ *   h[i,j]     = Abar[i,j]*h[i,j-1]  + vv[i,j]                   h[i,-1]  = 0
+ *   y[i,j]    += C[n,i,j]*h[i,j]
+ *
  * Orientations (READING of "reverse scans" in [PN 局限与展望] and "四象限" in [J 7.4]):
  * an orientation flips the map in H and/or W, runs the scan above from its own corner
  * with its own B_k, C_k (stored in the original, unflipped coordinates), and its output is
@@ -44,7 +51,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-#define ORACLE_VERSION 1
+#define ORACLE_VERSION 2
 
 /* bf16 bits -> double, exact (a bf16 value is the top 16 bits of an IEEE fp32 value). */
 static double bf16_to_double(uint16_t v)
@@ -67,6 +74,7 @@ typedef struct {
     const void *x, *delta, *B, *C;
     const float *A, *Dskip;
     int batch, channels, H, W, N, K, is_bf16;
+    int vfirst;                                     /* bit 4 of the mask: vertical first */
 } problem;
 
 /* Orientation number (0..3) of the k-th set bit of the mask, or -1. */
@@ -92,6 +100,7 @@ static int orientation_of(unsigned mask, int k)
 static void scan_one_orientation(const problem *p, int b, int d, int k, int orient,
                                  int rows, int cols, double *yacc, double *hcol)
 {
+    const int vfirst = p->vfirst;
     const int H = p->H, W = p->W, N = p->N, K = p->K;
     const int flipW = orient & 1, flipH = (orient >> 1) & 1;
     const size_t map = ((size_t)b * p->channels + d) * (size_t)H * W;
@@ -111,9 +120,15 @@ static void scan_one_orientation(const problem *p, int b, int d, int k, int orie
                 const double Bv = load(p->B, bc + pos, p->is_bf16);
                 const double Cv = load(p->C, bc + pos, p->is_bf16);
                 const double abar = exp(dl * An);          /* Abar = exp(delta*A)   */
-                hh = abar * hh + (dl * Bv) * xv;           /* horizontal, [J 4.5(1)] */
-                hcol[jj] = abar * hcol[jj] + hh;           /* vertical,   [J 4.5(2)] */
-                yacc[pos] += Cv * hcol[jj];                /* y = C h,    [J 4.5(2)] */
+                if (!vfirst) {
+                    hh = abar * hh + (dl * Bv) * xv;       /* horizontal, [J 4.5(1)] */
+                    hcol[jj] = abar * hcol[jj] + hh;       /* vertical,   [J 4.5(2)] */
+                    yacc[pos] += Cv * hcol[jj];            /* y = C h,    [J 4.5(2)] */
+                } else {
+                    hcol[jj] = abar * hcol[jj] + (dl * Bv) * xv;   /* vertical first  */
+                    hh = abar * hh + hcol[jj];             /* then horizontal       */
+                    yacc[pos] += Cv * hh;                  /* y = C h               */
+                }
             }
         }
     }
@@ -125,7 +140,7 @@ static int check(const problem *p, unsigned mask)
         return -1;
     if (p->batch < 1 || p->channels < 1 || p->H < 1 || p->W < 1 || p->N < 1)
         return -2;
-    if (mask == 0 || (mask & ~0xFu))
+    if ((mask & 0xFu) == 0 || (mask & ~0x1Fu))
         return -4;
     return 0;
 }
@@ -137,6 +152,7 @@ static void init_problem(problem *p, const void *x, const void *delta, const flo
     p->x = x; p->delta = delta; p->A = A; p->B = B; p->C = C; p->Dskip = Dskip;
     p->batch = batch; p->channels = channels; p->H = H; p->W = W; p->N = N;
     p->is_bf16 = is_bf16;
+    p->vfirst = (mask >> 4) & 1u;
     p->K = 0;
     for (int o = 0; o < 4; ++o)
         p->K += (mask >> o) & 1u;

@@ -33,6 +33,7 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 struct Shape {
   int batch, channels, H, W, N, K;
   bool bf16, out_f32;
+  bool vfirst;                 // vertical scan first (SCAN2D_VFIRST)
   unsigned orient;             // 4-bit orientation mask
   size_t in_elem, out_elem;    // bytes per element of x/delta/B/C and of y
   size_t xy_count, bc_count;   // elements of x (= y) and of B (= C)
@@ -54,6 +55,7 @@ int check_shape(int batch, int channels, int H, int W, int N, unsigned flags, Sh
   s->batch = batch; s->channels = channels; s->H = H; s->W = W; s->N = N; s->K = K;
   s->bf16 = (flags & SCAN2D_BF16) != 0;
   s->out_f32 = !s->bf16 || (flags & SCAN2D_OUT_F32) != 0;
+  s->vfirst = (flags & SCAN2D_VFIRST) != 0;
   s->orient = orient;
   s->in_elem = s->bf16 ? 2 : 4;
   s->out_elem = s->out_f32 ? 4 : 2;
@@ -486,6 +488,7 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
   prm.timeout_ns = kTimeoutNs;
   prm.yacc_stride = cp.yacc_stride;
   prm.orient_split = cp.orient_split;
+  prm.vfirst = s.vfirst ? 1 : 0;
   prm.out_f32 = s.out_f32 ? 1 : 0;
   prm.vec_store = (W % 4 == 0) && aligned(y, s.out_f32 ? 16 : 8);
 

@@ -96,6 +96,7 @@ struct Params {
   int orient_k[4];          // index of the orientation's B_k, C_k
   int mode;
   int yacc_stride;          // kSmemMulti: floats per channel in shared memory
+  int vfirst;               // 1: vertical scan first, then the horizontal one (carried across strips)
   int orient_split;         // kSmemMulti: 2 when the block's two chain slots walk every other
                             // orientation of the same channels (else 1)
   int vec_store;            // rows of y are aligned for 4-column vector stores
@@ -835,7 +836,9 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
 
       // ---- (3) the strip's columns of this row, two adjacent columns at a time -------------
       float2 acc[NP][G];
-      auto vec_group = [&](int vg, bool rev) {
+      // vf: vertical-first order.  The carried chain is then the second (horizontal) scan of
+      // the vertical state, and the output contracts that chain's state.
+      auto vec_group = [&](int vg, bool rev, bool vf) {
         uint4 xv[G], dv[G], bv[NG], cv[NG];
 #pragma unroll
         for (int c = 0; c < G; ++c) {
@@ -862,32 +865,42 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
               const float2 arg = __fmul2_rn(d2, A2[c][g]);
               const float2 a = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
               const float2 uu = __fmul2_rn(dx, Elem<Tin>::pair(bv[g], kp));
+              if (vf) v[pp][c][g] = __ffma2_rn(a, v[pp][c][g], uu);          // vertical first
+              const float2 in2 = vf ? v[pp][c][g] : uu;                       // input of the chain
               float2 h2;
               if (!rev) {
-                h2.x = fmaf(a.x, hh[c][g], uu.x);
-                h2.y = fmaf(a.y, h2.x, uu.y);
+                h2.x = fmaf(a.x, hh[c][g], in2.x);
+                h2.y = fmaf(a.y, h2.x, in2.y);
                 hh[c][g] = h2.y;
               } else {
-                h2.y = fmaf(a.y, hh[c][g], uu.y);
-                h2.x = fmaf(a.x, h2.y, uu.x);
+                h2.y = fmaf(a.y, hh[c][g], in2.y);
+                h2.x = fmaf(a.x, h2.y, in2.x);
                 hh[c][g] = h2.x;
               }
-              v[pp][c][g] = __ffma2_rn(a, v[pp][c][g], h2);
-              a_acc = __ffma2_rn(Elem<Tin>::pair(cv[g], kp), v[pp][c][g], a_acc);
+              if (!vf) v[pp][c][g] = __ffma2_rn(a, v[pp][c][g], h2);         // then vertical
+              a_acc = __ffma2_rn(Elem<Tin>::pair(cv[g], kp), vf ? h2 : v[pp][c][g], a_acc);
             }
             acc[pp][c] = a_acc;
           }
         }
       };
       float own_prev[E / 4];                                 // the pending row, reduced
-      if (!flipW) {
+      if (!flipW && !p.vfirst) {
         reduce_row(pacc, own_prev);
 #pragma unroll
-        for (int vg = 0; vg < NVEC; ++vg) vec_group(vg, false);
+        for (int vg = 0; vg < NVEC; ++vg) vec_group(vg, false, false);
+      } else if (!p.vfirst) {
+        reduce_row(pacc, own_prev);
+#pragma unroll
+        for (int vg = NVEC - 1; vg >= 0; --vg) vec_group(vg, true, false);
+      } else if (!flipW) {
+        reduce_row(pacc, own_prev);
+#pragma unroll
+        for (int vg = 0; vg < NVEC; ++vg) vec_group(vg, false, true);
       } else {
         reduce_row(pacc, own_prev);
 #pragma unroll
-        for (int vg = NVEC - 1; vg >= 0; --vg) vec_group(vg, true);
+        for (int vg = NVEC - 1; vg >= 0; --vg) vec_group(vg, true, true);
       }
 
       // ---- (4) carry-out to the next strip, as early as possible -----------------------------

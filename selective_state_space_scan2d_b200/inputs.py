@@ -45,6 +45,7 @@ class Workload:
     wsi_mask: bool = False
     random_A: bool = False
     dskip: bool = True
+    vfirst: bool = False               # scan order: vertical first (not an input, a flag)
 
     @property
     def K(self) -> int:
@@ -152,4 +153,4 @@ def make_inputs(w: Workload | str, seed: int = 0) -> dict:
     elif w.dtype != "f32":
         raise ValueError(w.dtype)
     return dict(x=x, delta=delta, A=np.ascontiguousarray(A, dtype=np.float32), B=B, C=C,
-                Dskip=Dskip, workload=w, orient_mask=w.orient_mask)
+                Dskip=Dskip, workload=w, orient_mask=w.orient_mask, vfirst=w.vfirst)

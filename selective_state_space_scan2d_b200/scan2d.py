@@ -45,6 +45,7 @@ _lib.scan2d_version.restype = _i
 # flags (include/scan2d.h)
 SCAN2D_BF16 = 0x1
 SCAN2D_OUT_F32 = 0x2
+SCAN2D_VFIRST = 0x8
 SCAN2D_OR_TL = 0x10
 SCAN2D_OR_TR = 0x20
 SCAN2D_OR_BL = 0x40
@@ -67,11 +68,14 @@ def scan2d_version() -> int:
     return int(_lib.scan2d_version())
 
 
-def flags_for(bf16: bool, orient_mask: int = 1, out_f32: bool = False) -> int:
-    """Flag word for an element type and a 4-bit orientation mask (bit0 TL .. bit3 BR)."""
+def flags_for(bf16: bool, orient_mask: int = 1, out_f32: bool = False, vfirst: bool = False) -> int:
+    """Flag word for an element type, a 4-bit orientation mask (bit0 TL .. bit3 BR) and the
+    scan order (vfirst: vertical scan first)."""
     f = (SCAN2D_BF16 if bf16 else 0) | ((orient_mask & 0xF) << 4)
     if out_f32:
         f |= SCAN2D_OUT_F32
+    if vfirst:
+        f |= SCAN2D_VFIRST
     return f
 
 

@@ -40,6 +40,12 @@ CASES = {
     "bf16_k4_split_plain": ("vision", dict(batch=1, channels=8, H=9, W=44)),
     "bf16_k3_split_plain": ("vision", dict(batch=2, channels=8, H=11, W=41, orient_mask=0b0111)),
     "f32_k2_split_tma": ("tiny", dict(batch=1, channels=8, N=16, H=12, W=48, orient_mask=0b0011)),
+    # vertical-then-horizontal scan order
+    "f32_vfirst_chain_tma": ("tiny", dict(batch=1, channels=8, N=16, H=13, W=200, vfirst=True)),
+    "f32_vfirst_global_ring": ("tiny", dict(batch=1, channels=16, N=16, H=21, W=1056, vfirst=True)),
+    "f32_vfirst_plain_flips": ("tiny", dict(batch=1, channels=9, N=16, H=11, W=45, orient_mask=0b1010, vfirst=True)),
+    "bf16_vfirst_k4_split": ("vision", dict(batch=1, channels=8, H=20, W=56, vfirst=True)),
+    "bf16_vfirst_k4_global": ("vision", dict(batch=1, channels=8, H=14, W=300, vfirst=True)),
 }
 for n in (1, 3, 5, 8, 12, 17, 32, 33, 64):
     CASES[f"N{n}"] = ("tiny", dict(batch=1, channels=9, N=n, H=9, W=23))

@@ -29,7 +29,7 @@ def run_gpu(d, flags=None, stream=None):
     from selective_state_space_scan2d_b200 import scan2d
     t = to_torch(d)
     if flags is None:
-        flags = scan2d.flags_for(d["x"].dtype == np.uint16, d["orient_mask"])
+        flags = scan2d.flags_for(d["x"].dtype == np.uint16, d["orient_mask"], vfirst=d.get("vfirst", False))
     return scan2d.scan2d_fwd(t["x"], t["delta"], t["A"], t["B"], t["C"], t["Dskip"],
                              flags=flags, stream=stream)
 

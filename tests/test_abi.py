@@ -52,6 +52,7 @@ def test_binding_constants_match_header(lib):
                  "SCAN2D_OR_BL", "SCAN2D_OR_BR"):
         assert getattr(lib, name) == m[name], name
     assert lib.SCAN2D_E_SCRATCH == m["SCAN2D_E_SCRATCH"]
+    assert lib.SCAN2D_VFIRST == m["SCAN2D_VFIRST"]
     assert lib.SCAN2D_NOALLOC_SCRATCH_BYTES == m["SCAN2D_NOALLOC_SCRATCH_BYTES"]
     assert lib.flags_for(True, 0xF, out_f32=True) == (m["SCAN2D_BF16"] | m["SCAN2D_OUT_F32"] | m["SCAN2D_OR_ALL"])
 

@@ -16,8 +16,9 @@ if not torch.cuda.is_available():
 
 
 def _oracle_full(oracle_mod, d, mask=None):
-    return oracle_mod.scan2d_fwd(d["x"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"],
-                                 d["orient_mask"] if mask is None else mask)
+    if mask is None:
+        mask = d["orient_mask"] | (0x10 if d.get("vfirst") else 0)   # oracle bit 4: vertical first
+    return oracle_mod.scan2d_fwd(d["x"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"], mask)
 
 
 def _check_full(oracle_mod, d, flags=None, mask=None):
@@ -149,3 +150,19 @@ def test_workspace_reuse_across_shapes(oracle_mod):
     from selective_state_space_scan2d_b200 import scan2d
     assert scan2d.scan2d_get_device_error(s) == 0
     assert_parity(y_to_f64(y), _oracle_full(oracle_mod, big), TOL["f32"], "reuse")
+
+
+def test_full_size_vfirst_giga_shape(oracle_mod):
+    """Vertical-then-horizontal order at the giga shape, in the launch configuration of the
+    default order (the flag changes only the math inside a row)."""
+    w = inputs.WORKLOADS["giga"].scaled(vfirst=True)
+    d = inputs.make_inputs(w, seed=2)
+    y = run_gpu(d)
+    torch.cuda.synchronize()
+    from selective_state_space_scan2d_b200 import scan2d
+    assert scan2d.scan2d_get_device_error() == 0
+    maps = [(0, 3), (0, 126)]
+    ym = oracle_mod.scan2d_maps(d["x"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"], maps, 1 | 0x10)
+    for m, (b, ch) in enumerate(maps):
+        got = y[b, ch].to("cpu", torch.float64).numpy()
+        assert_parity(got, ym[m], TOL["f32"], f"vertical-first map {(b, ch)}")

@@ -74,6 +74,27 @@ def linsolve_map(x, dl, A, B, C, D):
     return y.reshape(H, W)
 
 
+def closed_form_map_vfirst(x, dl, A, B, C, D):
+    """Vertical-then-horizontal order, brute force: the path from (i', j') runs down column
+    j' to row i, then right along row i:
+    h[i,j] = sum prod_{l=j'+1..j} Abar[i,l] * prod_{k=i'+1..i} Abar[k,j'] * Bbar x[i',j']."""
+    H, W = x.shape
+    y = D * x.copy()
+    for n in range(A.shape[0]):
+        a = np.exp(dl * A[n])
+        u = dl * B[n] * x
+        for i in range(H):
+            for j in range(W):
+                s = 0.0
+                for jp in range(j + 1):
+                    right = np.prod(a[i, jp + 1:j + 1])
+                    for ip in range(i + 1):
+                        down = np.prod(a[ip + 1:i + 1, jp])
+                        s += right * down * u[ip, jp]
+                y[i, j] += C[n, i, j] * s
+    return y
+
+
 def recurrence_1d(a, u):
     """Textbook 1D selective recurrence h_t = a_t h_{t-1} + u_t, h_{-1} = 0."""
     h = np.zeros_like(u)
@@ -234,6 +255,35 @@ def pin_orientations(oracle_mod, lib=None):
     np.testing.assert_allclose(y2, ysum, rtol=1e-12, atol=1e-12)
 
 
+VFIRST = 0x10     # oracle mask bit: vertical-then-horizontal scan order
+
+
+def pin_vfirst_closed_form(oracle_mod, lib=None):
+    """Vertical-first order ("scan order" ablation, papernotes.org): brute-force path sums."""
+    for (H, W, N, seed) in [(6, 5, 3, 11), (4, 8, 2, 12)]:
+        d = _small(H=H, W=W, N=N, channels=2, batch=1, seed=seed, random_A=True)
+        y = _fwd(oracle_mod, d, lib, mask=1 | VFIRST)
+        for ch in range(2):
+            np.testing.assert_allclose(y[0, ch], closed_form_map_vfirst(*_map_args(d, 0, ch)),
+                                       rtol=1e-12, atol=1e-12)
+
+
+def pin_vfirst_transpose(oracle_mod, lib=None):
+    """Vertical-first on a map = horizontal-first on the transposed map, transposed back
+    (flip W and flip H trade places under the transpose)."""
+    d = _small(H=5, W=7, N=3, channels=2, batch=2, seed=13, random_A=True)
+    T = lambda a: np.swapaxes(a, -1, -2).copy()
+    for o, o_t in ((0, 0), (1, 2), (2, 1), (3, 3)):          # TL, TR, BL, BR -> TL, BL, TR, BR
+        y = _fwd(oracle_mod, d, lib, mask=(1 << o) | VFIRST)
+        yt = oracle_mod.scan2d_fwd(T(d["x"]), T(d["delta"]), d["A"], T(d["B"]), T(d["C"]), d["Dskip"],
+                                   1 << o_t, lib=lib)
+        np.testing.assert_allclose(y, T(yt), rtol=1e-12, atol=1e-12)
+    # the order matters when Abar varies (the two orders are different operators)
+    yh = _fwd(oracle_mod, d, lib, mask=1)
+    yv = _fwd(oracle_mod, d, lib, mask=1 | VFIRST)
+    assert np.max(np.abs(yh - yv)) > 1e-6
+
+
 def pin_points_and_maps(oracle_mod, lib=None):
     d = _small(H=9, W=11, N=3, channels=3, batch=2, seed=8, orient_mask=0b1101)
     y = _fwd(oracle_mod, d, lib)
@@ -248,7 +298,8 @@ def pin_points_and_maps(oracle_mod, lib=None):
 
 
 PINS = [pin_closed_form, pin_linsolve, pin_manhattan_constant, pin_golden_3x3,
-        pin_1d_reduction, pin_linearity_and_special, pin_orientations, pin_points_and_maps]
+        pin_1d_reduction, pin_linearity_and_special, pin_orientations, pin_vfirst_closed_form,
+        pin_vfirst_transpose, pin_points_and_maps]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -302,6 +353,9 @@ MUTATIONS = {
                                    "static double hh; if (ii == 0) hh = 0.0;"),
     "state_index_off_by_one": ("const double An = (double)p->A[(size_t)d * N + n];",
                                "const double An = (double)p->A[(size_t)d * N + (n + 1) % N];"),
+    "vfirst_ignored": ("const int vfirst = p->vfirst;", "const int vfirst = 0;"),
+    "vfirst_vertical_without_decay": ("hcol[jj] = abar * hcol[jj] + (dl * Bv) * xv;",
+                                      "hcol[jj] = hcol[jj] + (dl * Bv) * xv;"),
 }
 
 
