@@ -72,8 +72,9 @@ struct Variant {
   size_t tile_bytes_tma;      // one staged tile of kTileRows strip rows (TMA path)
   size_t tile_bytes_plain;    // one staged strip row (plain-load path)
   size_t carry_slot_bytes;    // one carry row of a warp
-  KernelFn fn_tma, fn_plain;
-  KernelFn fn_tma16, fn_plain16;   // up to 16 warps per block (one channel per lane only)
+  // [scan order: 0 horizontal first, 1 vertical first]
+  KernelFn fn_tma[2], fn_plain[2];
+  KernelFn fn_tma16[2], fn_plain16[2];   // up to 16 warps per block (one channel per lane only)
 };
 
 template <typename Tin, int NG, int G, int CMAX>
@@ -82,10 +83,14 @@ Variant make_variant() {
   using LP = Layout<Tin, NG, G, CMAX, 1>;
   Variant v{NG, G, CMAX, static_cast<size_t>(LT::TILE_BYTES), static_cast<size_t>(LP::TILE_BYTES),
             static_cast<size_t>(LP::CARRY_SLOT_BYTES),
-            scan2d_kernel<Tin, NG, G, CMAX, true>, scan2d_kernel<Tin, NG, G, CMAX, false>, nullptr, nullptr};
+            {scan2d_kernel<Tin, NG, G, CMAX, true, kMaxWarps, false>, scan2d_kernel<Tin, NG, G, CMAX, true, kMaxWarps, true>},
+            {scan2d_kernel<Tin, NG, G, CMAX, false, kMaxWarps, false>, scan2d_kernel<Tin, NG, G, CMAX, false, kMaxWarps, true>},
+            {nullptr, nullptr}, {nullptr, nullptr}};
   if constexpr (G == 1) {
-    v.fn_tma16 = scan2d_kernel<Tin, NG, G, CMAX, true, kMaxWarpsSplit>;
-    v.fn_plain16 = scan2d_kernel<Tin, NG, G, CMAX, false, kMaxWarpsSplit>;
+    v.fn_tma16[0] = scan2d_kernel<Tin, NG, G, CMAX, true, kMaxWarpsSplit, false>;
+    v.fn_tma16[1] = scan2d_kernel<Tin, NG, G, CMAX, true, kMaxWarpsSplit, true>;
+    v.fn_plain16[0] = scan2d_kernel<Tin, NG, G, CMAX, false, kMaxWarpsSplit, false>;
+    v.fn_plain16[1] = scan2d_kernel<Tin, NG, G, CMAX, false, kMaxWarpsSplit, true>;
   }
   return v;
 }
@@ -309,7 +314,7 @@ CallPlan plan_call(const Shape& s, bool tma, bool cluster_ok, int nsm) {
       const size_t split_smem = sizeof(float) * p1.cpw * stride + 2 * (p1.tile_smem + p1.carry_smem);
       // (up to 4 states per lane: the 16-warp variants get 128 registers a thread)
       if (p1.chains_per_block == 1 && 2 * p1.wpc <= kMaxWarpsSplit && split_smem <= kSmemBudgetSplit &&
-          p1.var.fn_tma16 != nullptr && ng <= 4) {
+          p1.var.fn_tma16[0] != nullptr && ng <= 4) {
         p1.tile_smem *= 2;
         p1.carry_smem *= 2;
         p1.chains_per_block = 2;
@@ -470,12 +475,13 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
   }
   // a chain's blocks share distributed shared memory when such a cluster fits on the device
   if (cp.link == kLinkCluster &&
-      !cluster_worth_it(tma ? cp.pl.var.fn_tma : cp.pl.var.fn_plain, cp.pl.warps * 32, cp.smem, cp.pl.nseg,
+      !cluster_worth_it(tma ? cp.pl.var.fn_tma[s.vfirst ? 1 : 0] : cp.pl.var.fn_plain[s.vfirst ? 1 : 0], cp.pl.warps * 32, cp.smem, cp.pl.nseg,
                         cp.pl.n_chains))
     cp = plan_call(s, tma, false, nsm);
   const Plan& pl = cp.pl;
-  const KernelFn fn = cp.orient_split > 1 ? (tma ? pl.var.fn_tma16 : pl.var.fn_plain16)
-                                         : (tma ? pl.var.fn_tma : pl.var.fn_plain);
+  const int vf = s.vfirst ? 1 : 0;
+  const KernelFn fn = cp.orient_split > 1 ? (tma ? pl.var.fn_tma16[vf] : pl.var.fn_plain16[vf])
+                                         : (tma ? pl.var.fn_tma[vf] : pl.var.fn_plain[vf]);
 
   Params prm;
   std::memset(&prm, 0, sizeof prm);
@@ -488,7 +494,6 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
   prm.timeout_ns = kTimeoutNs;
   prm.yacc_stride = cp.yacc_stride;
   prm.orient_split = cp.orient_split;
-  prm.vfirst = s.vfirst ? 1 : 0;
   prm.out_f32 = s.out_f32 ? 1 : 0;
   prm.vec_store = (W % 4 == 0) && aligned(y, s.out_f32 ? 16 : 8);
 

@@ -96,7 +96,6 @@ struct Params {
   int orient_k[4];          // index of the orientation's B_k, C_k
   int mode;
   int yacc_stride;          // kSmemMulti: floats per channel in shared memory
-  int vfirst;               // 1: vertical scan first, then the horizontal one (carried across strips)
   int orient_split;         // kSmemMulti: 2 when the block's two chain slots walk every other
                             // orientation of the same channels (else 1)
   int vec_store;            // rows of y are aligned for 4-column vector stores
@@ -413,7 +412,7 @@ __host__ __device__ constexpr size_t carry_ring_bytes(int warps) {
 }
 
 // ---- the kernel ------------------------------------------------------------------------------
-template <typename Tin, int NG, int G, int CMAX, bool TMA, int MAXW = kMaxWarps>
+template <typename Tin, int NG, int G, int CMAX, bool TMA, int MAXW = kMaxWarps, bool VF = false>
 __global__ void __launch_bounds__(MAXW * 32, 1)
 scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps tm) {
   constexpr int R = TMA ? kTileRows : 1;                     // rows per staged tile
@@ -444,9 +443,11 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   // two warps of a sub-partition take adjacent strips (strip s on warp s/2 + 4 (s % 2)): a warp
   // then computes while its partner waits for the carry it is about to hand over, instead of
   // both computing (or both waiting) at the same time.
-  const bool pair_map = p.wpc == 8 && p.chains_per_block == 1;
+  const bool pair_map = MAXW == kMaxWarps && p.wpc == 8 && p.chains_per_block == 1;
   auto warp_of = [&](int ws) { return pair_map ? (ws >> 1) + 4 * (ws & 1) : slot * p.wpc + ws; };
   const int w = is_compute ? (pair_map ? 2 * (warp & 3) + (warp >> 2) : warp - slot * p.wpc) : 0;  // strip
+  const int next_warp = warp_of(w + 1);                      // warps of the neighbouring strips
+  const int prev_warp = warp_of(w - 1);
   const int cg = lane >> 2;                 // channel group
   const int q = lane & 3;                   // state group
   const bool cluster = p.link == kLinkCluster;
@@ -636,7 +637,7 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   }
 
   // where this warp's carries go: the next warp of this block, or warp 0 of the next block
-  const uint32_t next_full0 = smem_u32(&s_full[next_local ? warp_of(w + 1) : 0][0]);
+  const uint32_t next_full0 = smem_u32(&s_full[next_local ? next_warp : 0][0]);
   const uint32_t my_empty0 = smem_u32(&s_empty[warp][0]);
   uint32_t next_ring_cl = 0, next_full_cl = 0, prev_empty_cl = 0;
   if (cluster) {
@@ -826,7 +827,7 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
 #pragma unroll
           for (int g = 0; g < NG; ++g) hh[c][g] = in[c * NG + g];
         // free the slot (a slot filled from another block is freed once its values are used)
-        if (!left_remote) mbar_arrive_local(smem_u32(&s_empty[warp_of(w - 1)][cs]));
+        if (!left_remote) mbar_arrive_local(smem_u32(&s_empty[prev_warp][cs]));
       } else {
 #pragma unroll
         for (int c = 0; c < G; ++c)
@@ -885,22 +886,14 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
         }
       };
       float own_prev[E / 4];                                 // the pending row, reduced
-      if (!flipW && !p.vfirst) {
+      if (!flipW) {
         reduce_row(pacc, own_prev);
 #pragma unroll
-        for (int vg = 0; vg < NVEC; ++vg) vec_group(vg, false, false);
-      } else if (!p.vfirst) {
-        reduce_row(pacc, own_prev);
-#pragma unroll
-        for (int vg = NVEC - 1; vg >= 0; --vg) vec_group(vg, true, false);
-      } else if (!flipW) {
-        reduce_row(pacc, own_prev);
-#pragma unroll
-        for (int vg = 0; vg < NVEC; ++vg) vec_group(vg, false, true);
+        for (int vg = 0; vg < NVEC; ++vg) vec_group(vg, false, VF);
       } else {
         reduce_row(pacc, own_prev);
 #pragma unroll
-        for (int vg = NVEC - 1; vg >= 0; --vg) vec_group(vg, true, true);
+        for (int vg = NVEC - 1; vg >= 0; --vg) vec_group(vg, true, VF);
       }
 
       // ---- (4) carry-out to the next strip, as early as possible -----------------------------
@@ -916,7 +909,7 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
 #pragma unroll
           for (int g = 0; g < NG; ++g) out[c * NG + g] = hh[c][g];
         if (next_local) {
-          float4* dst = reinterpret_cast<float4*>(carry_slot(warp_of(w + 1), cs)) + lane * (L::CARRY_PAD / 4);
+          float4* dst = reinterpret_cast<float4*>(carry_slot(next_warp, cs)) + lane * (L::CARRY_PAD / 4);
 #pragma unroll
           for (int k4 = 0; k4 < L::CARRY_PAD / 4; ++k4)
             dst[k4] = make_float4(out[4 * k4], out[4 * k4 + 1], out[4 * k4 + 2], out[4 * k4 + 3]);

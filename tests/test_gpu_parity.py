@@ -166,3 +166,27 @@ def test_full_size_vfirst_giga_shape(oracle_mod):
     for m, (b, ch) in enumerate(maps):
         got = y[b, ch].to("cpu", torch.float64).numpy()
         assert_parity(got, ym[m], TOL["f32"], f"vertical-first map {(b, ch)}")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_unaligned_buffers_use_plain_loads(oracle_mod, dtype):
+    """Buffers that start one element past a 16-byte boundary cannot be staged by TMA: the
+    call takes the plain-load path for a shape that would otherwise use TMA."""
+    from selective_state_space_scan2d_b200 import scan2d
+    name = "small" if dtype == "bf16" else "tiny"
+    w = workload(name, batch=1, channels=8, N=16, H=9, W=64)
+    d = inputs.make_inputs(w, seed=8)
+    t = to_torch(d)
+
+    def shifted(a):               # same values, storage starting one element later
+        buf = torch.empty(a.numel() + 1, dtype=a.dtype, device=a.device)
+        v = buf[1:].view(a.shape)
+        v.copy_(a)
+        return v
+    s = {k: (shifted(v) if k in ("x", "delta", "B", "C") else v) for k, v in t.items()}
+    assert s["x"].data_ptr() % 16 != 0
+    y = scan2d.scan2d_fwd(s["x"], s["delta"], s["A"], s["B"], s["C"], s["Dskip"],
+                          flags=scan2d.flags_for(dtype == "bf16", 1))
+    torch.cuda.synchronize()
+    assert scan2d.scan2d_get_device_error() == 0
+    assert_parity(y_to_f64(y), _oracle_full(oracle_mod, d), TOL[dtype], f"unaligned {dtype}")
