@@ -1,4 +1,4 @@
-"""fp64 CPU oracle of the 2D selective-scan forward (2DMamba), as a ctypes binding.
+"""fp64 CPU oracle of the 2D selective-scan forward (2DMamba) and its gradients, as a ctypes binding.
 
 TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU
 baseline leg of ``bench.py`` may import this package.  The product path (the CUDA
@@ -57,6 +57,9 @@ def load_library(path: str | None = None):
     lib.scan2d_oracle_maps.restype = i
     lib.scan2d_oracle_points.argtypes = common + [ip, i]
     lib.scan2d_oracle_points.restype = i
+    lib.scan2d_oracle_bwd.argtypes = [vp, vp, fp, vp, vp, fp, dp, dp, dp, dp, dp, dp, dp,
+                                      i, i, i, i, i, i, u, i]
+    lib.scan2d_oracle_bwd.restype = i
     lib.scan2d_oracle_version.argtypes = []
     lib.scan2d_oracle_version.restype = i
     if path is None:
@@ -139,6 +142,29 @@ def scan2d_points(x, delta, A, B, C, Dskip, points, orient_mask: int = 1, lib=No
     if rc:
         raise RuntimeError(f"oracle error {rc}")
     return y
+
+
+def scan2d_bwd(x, delta, A, B, C, Dskip, dy, orient_mask: int = 1, majorant: bool = False,
+               lib=None) -> dict:
+    """fp64 gradients of sum(dy * y) with respect to every input: a dict with dx, ddelta
+    (batch, channels, H, W), dA (channels, N), dB, dC (batch, K, N, H, W) and dDskip
+    (channels,).  majorant=True returns, for each output, the sum of the magnitudes of the
+    terms that make it up (the scale of any evaluation's rounding error)."""
+    x, delta, A, B, C, Dskip, dims = _prepare(x, delta, A, B, C, Dskip, orient_mask)
+    batch, channels, H, W, N, _ = dims
+    K = B.shape[1]
+    dy = np.ascontiguousarray(dy, dtype=np.float64)
+    if dy.shape != x.shape:
+        raise ValueError("dy must have the shape of x")
+    out = {"dx": np.empty(x.shape), "ddelta": np.empty(x.shape), "dA": np.empty((channels, N)),
+           "dB": np.empty((batch, K, N, H, W)), "dC": np.empty((batch, K, N, H, W)),
+           "dDskip": np.empty(channels)}
+    rc = _load(lib).scan2d_oracle_bwd(_ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(Dskip),
+                                   _ptr(dy), *(_ptr(out[k]) for k in ("dx", "ddelta", "dA", "dB", "dC", "dDskip")),
+                                   *dims, orient_mask, int(bool(majorant)))
+    if rc:
+        raise RuntimeError(f"oracle error {rc}")
+    return out
 
 
 def version() -> int:

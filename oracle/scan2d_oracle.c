@@ -1,5 +1,6 @@
 /*
- * scan2d_oracle.c -- plain, slow, fp64 reference of the 2D selective-scan forward.
+ * scan2d_oracle.c -- plain, slow, fp64 reference of the 2D selective-scan forward and of
+ * its gradients.
  *
  * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the CPU-baseline
  * leg of the benchmark may load this code.  The product path (the CUDA library) shares
@@ -51,7 +52,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-#define ORACLE_VERSION 2
+#define ORACLE_VERSION 3
 
 /* bf16 bits -> double, exact (a bf16 value is the top 16 bits of an IEEE fp32 value). */
 static double bf16_to_double(uint16_t v)
@@ -272,6 +273,158 @@ int scan2d_oracle_points(const void *x, const void *delta, const float *A, const
     }
     free(hcol);
     free(yacc);
+    return 0;
+}
+
+/*
+ * Gradients of the forward above (the pages give no backward pass; these are the plain
+ * chain-rule adjoints of the two recurrences, READING: the training gradient of y).
+ *
+ * For a cotangent dy (fp64, (batch, channels, H, W)) they are the derivatives of
+ *   L = sum_{b,d,i,j} dy[b,d,i,j] * y[b,d,i,j]
+ * with respect to x, delta (same layout as x), A (channels, N), B and C
+ * ((batch, K, N, H, W), summed over the channels that share them) and Dskip (channels).
+ *
+ * Writing s1 for the first scan's state and s2 for the second's (s1 = hh, s2 = h in the
+ * horizontal-first order; s1 = vv, s2 = h vertical-first), the adjoint of s2 runs the
+ * second scan backwards and the adjoint of s1 runs the first scan backwards:
+ *   g2[p] = C[p]*dy[p] + Abar[p+e2]*g2[p+e2]     (e2 = the second scan's step)
+ *   g1[p] = g2[p]      + Abar[p+e1]*g1[p+e1]     (e1 = the first scan's step)
+ *   dL/dAbar[p] = g2[p]*s2[p-e2] + g1[p]*s1[p-e1],   dL/du[p] = g1[p],  u = delta*B*x
+ * and then, with Abar = exp(delta*A):
+ *   dx     += g1*delta*B                dB += g1*delta*x
+ *   ddelta += dAbar*Abar*A + g1*B*x      dC += dy*s2
+ *   dA     += dAbar*Abar*delta           dDskip += dy*x,  dx += Dskip*dy (once).
+ *
+ * majorant != 0 replaces every stored value by its magnitude and the factor A by |A|
+ * (Abar itself keeps exp(delta*A)).  Every term of every sum is then non-negative, so
+ * each output is the sum of the magnitudes of the terms that make up the true gradient:
+ * the scale against which the rounding error of any evaluation order is bounded.
+ */
+static double mag(double v, int majorant) { return majorant ? fabs(v) : v; }
+
+static void bwd_one_orientation(const problem *p, const double *dy, int b, int d, int k,
+                                int orient, int majorant, double *a, double *u, double *s1,
+                                double *s2, double *g1, double *g2, double *dx, double *ddelta,
+                                double *dA, double *dB, double *dC)
+{
+    const int H = p->H, W = p->W, N = p->N, K = p->K;
+    const int flipW = orient & 1, flipH = (orient >> 1) & 1;
+    const size_t HW = (size_t)H * W;
+    const size_t map = ((size_t)b * p->channels + d) * HW;
+/* scan-order (ii, jj) -> index into the per-map work arrays */
+#define AT(ii, jj) ((size_t)(ii) * W + (size_t)(jj))
+    for (int n = 0; n < N; ++n) {
+        const double An = (double)p->A[(size_t)d * N + n];
+        const double Af = majorant ? fabs(An) : An;
+        const size_t bc = (((size_t)b * K + k) * N + n) * HW;
+        /* forward states, kept whole */
+        for (int ii = 0; ii < H; ++ii)
+            for (int jj = 0; jj < W; ++jj) {
+                const int i = flipH ? H - 1 - ii : ii;     /* original position */
+                const int j = flipW ? W - 1 - jj : jj;
+                const size_t pos = (size_t)i * W + j, t = AT(ii, jj);
+                const double dl = mag(load(p->delta, map + pos, p->is_bf16), majorant);
+                const double xv = mag(load(p->x, map + pos, p->is_bf16), majorant);
+                const double Bv = mag(load(p->B, bc + pos, p->is_bf16), majorant);
+                a[t] = exp(dl * An);
+                u[t] = (dl * Bv) * xv;
+                if (!p->vfirst) {
+                    s1[t] = a[t] * (jj > 0 ? s1[AT(ii, jj - 1)] : 0.0) + u[t];
+                    s2[t] = a[t] * (ii > 0 ? s2[AT(ii - 1, jj)] : 0.0) + s1[t];
+                } else {
+                    s1[t] = a[t] * (ii > 0 ? s1[AT(ii - 1, jj)] : 0.0) + u[t];
+                    s2[t] = a[t] * (jj > 0 ? s2[AT(ii, jj - 1)] : 0.0) + s1[t];
+                }
+            }
+        /* adjoints, from the far corner back */
+        for (int ii = H - 1; ii >= 0; --ii)
+            for (int jj = W - 1; jj >= 0; --jj) {
+                const int i = flipH ? H - 1 - ii : ii;     /* original position */
+                const int j = flipW ? W - 1 - jj : jj;
+                const size_t pos = (size_t)i * W + j, t = AT(ii, jj);
+                const double gy = mag(dy[map + pos], majorant);
+                const double Cv = mag(load(p->C, bc + pos, p->is_bf16), majorant);
+                const int has_r = jj + 1 < W, has_d = ii + 1 < H;
+                if (!p->vfirst) {
+                    g2[t] = Cv * gy + (has_d ? a[AT(ii + 1, jj)] * g2[AT(ii + 1, jj)] : 0.0);
+                    g1[t] = g2[t] + (has_r ? a[AT(ii, jj + 1)] * g1[AT(ii, jj + 1)] : 0.0);
+                } else {
+                    g2[t] = Cv * gy + (has_r ? a[AT(ii, jj + 1)] * g2[AT(ii, jj + 1)] : 0.0);
+                    g1[t] = g2[t] + (has_d ? a[AT(ii + 1, jj)] * g1[AT(ii + 1, jj)] : 0.0);
+                }
+            }
+        /* what each position contributes */
+        double dA_n = 0.0;
+        for (int ii = 0; ii < H; ++ii)
+            for (int jj = 0; jj < W; ++jj) {
+                const int i = flipH ? H - 1 - ii : ii;     /* original position */
+                const int j = flipW ? W - 1 - jj : jj;
+                const size_t pos = (size_t)i * W + j, t = AT(ii, jj);
+                const double dl = mag(load(p->delta, map + pos, p->is_bf16), majorant);
+                const double xv = mag(load(p->x, map + pos, p->is_bf16), majorant);
+                const double Bv = mag(load(p->B, bc + pos, p->is_bf16), majorant);
+                const double gy = mag(dy[map + pos], majorant);
+                double s2_prev, s1_prev;                  /* s2[p - e2], s1[p - e1] */
+                if (!p->vfirst) {
+                    s2_prev = ii > 0 ? s2[AT(ii - 1, jj)] : 0.0;
+                    s1_prev = jj > 0 ? s1[AT(ii, jj - 1)] : 0.0;
+                } else {
+                    s2_prev = jj > 0 ? s2[AT(ii, jj - 1)] : 0.0;
+                    s1_prev = ii > 0 ? s1[AT(ii - 1, jj)] : 0.0;
+                }
+                const double dabar = g2[t] * s2_prev + g1[t] * s1_prev;
+                dx[map + pos] += g1[t] * dl * Bv;
+                ddelta[map + pos] += dabar * a[t] * Af + g1[t] * Bv * xv;
+                dA_n += dabar * a[t] * dl;
+                dB[bc + pos] += g1[t] * dl * xv;
+                dC[bc + pos] += gy * s2[t];
+            }
+        dA[(size_t)d * N + n] += dA_n;
+    }
+#undef AT
+}
+
+int scan2d_oracle_bwd(const void *x, const void *delta, const float *A, const void *B,
+                      const void *C, const float *Dskip, const double *dy, double *dx,
+                      double *ddelta, double *dA, double *dB, double *dC, double *dDskip,
+                      int batch, int channels, int H, int W, int N, int is_bf16,
+                      unsigned orient_mask, int majorant)
+{
+    problem p;
+    init_problem(&p, x, delta, A, B, C, Dskip, batch, channels, H, W, N, is_bf16, orient_mask);
+    int rc = check(&p, orient_mask);
+    if (rc)
+        return rc;
+    if (!dy || !dx || !ddelta || !dA || !dB || !dC || !dDskip)
+        return -1;
+    const size_t HW = (size_t)H * W;
+    const size_t nx = (size_t)batch * channels * HW, nbc = (size_t)batch * p.K * N * HW;
+    double *work = (double *)malloc(sizeof(double) * 6 * HW);
+    if (!work)
+        return -8;
+    memset(dx, 0, sizeof(double) * nx);
+    memset(ddelta, 0, sizeof(double) * nx);
+    memset(dA, 0, sizeof(double) * (size_t)channels * N);
+    memset(dB, 0, sizeof(double) * nbc);
+    memset(dC, 0, sizeof(double) * nbc);
+    memset(dDskip, 0, sizeof(double) * (size_t)channels);
+    for (int b = 0; b < batch; ++b)
+        for (int d = 0; d < channels; ++d) {
+            for (int k = 0; k < p.K; ++k)
+                bwd_one_orientation(&p, dy, b, d, k, orientation_of(orient_mask, k), majorant,
+                                    work, work + HW, work + 2 * HW, work + 3 * HW, work + 4 * HW,
+                                    work + 5 * HW, dx, ddelta, dA, dB, dC);
+            /* the skip term y += Dskip*x, added once */
+            const size_t map = ((size_t)b * channels + d) * HW;
+            const double Dd = Dskip ? mag((double)Dskip[d], majorant) : 0.0;
+            for (size_t pos = 0; pos < HW; ++pos) {
+                const double gy = mag(dy[map + pos], majorant);
+                dx[map + pos] += Dd * gy;
+                dDskip[d] += gy * mag(load(x, map + pos, is_bf16), majorant);
+            }
+        }
+    free(work);
     return 0;
 }
 

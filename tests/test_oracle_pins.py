@@ -297,9 +297,102 @@ def pin_points_and_maps(oracle_mod, lib=None):
     np.testing.assert_array_equal(ym[1], y[0, 1])
 
 
+# ----------------------------------------------------------------------------------------
+# gradients: the pages give no backward pass, so its oracle is pinned by routes that do not
+# share its adjoint recurrences (automatic differentiation, finite differences)
+# ----------------------------------------------------------------------------------------
+def torch_forward(x, dl, A, B, C, D, mask):
+    """The forward written once more with torch fp64 tensors, every (b, d, n) at once and a
+    Python loop over positions: orientations as flips of the inputs and of y."""
+    import torch
+    batch, ch, H, W = x.shape
+    y = D[None, :, None, None] * x
+    k = 0
+    for o in range(4):
+        if not (mask >> o) & 1:
+            continue
+        dims = ([3] if o & 1 else []) + ([2] if o & 2 else [])
+        fl = (lambda t: torch.flip(t, dims)) if dims else (lambda t: t)
+        xf, df = fl(x), fl(dl)
+        Bf, Cf = fl(B[:, k]), fl(C[:, k])                          # (batch, N, H, W)
+        a = torch.exp(df[:, :, None] * A[None, :, :, None, None])   # (batch, ch, N, H, W)
+        u = df[:, :, None] * Bf[:, None] * xf[:, :, None]
+        rows = []
+        col = [torch.zeros_like(a[..., 0, 0]) for _ in range(W)]
+        for i in range(H):
+            run = torch.zeros_like(a[..., 0, 0])
+            out = []
+            for j in range(W):
+                if not mask & 0x10:
+                    run = a[..., i, j] * run + u[..., i, j]           # horizontal
+                    col[j] = a[..., i, j] * col[j] + run            # vertical
+                    h = col[j]
+                else:
+                    col[j] = a[..., i, j] * col[j] + u[..., i, j]   # vertical first
+                    run = a[..., i, j] * run + col[j]
+                    h = run
+                out.append((Cf[:, None, :, i, j] * h).sum(2))
+            rows.append(torch.stack(out, -1))
+        y = y + fl(torch.stack(rows, -2))
+        k += 1
+    return y
+
+
+def _bwd(oracle_mod, d, dy, lib=None, mask=None, majorant=False):
+    return oracle_mod.scan2d_bwd(d["x"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"], dy,
+                                 d["orient_mask"] if mask is None else mask, majorant=majorant, lib=lib)
+
+
+def pin_bwd_autograd(oracle_mod, lib=None):
+    """Every gradient against torch's reverse-mode differentiation of the forward above,
+    both scan orders, one and four orientations; the majorant bounds each gradient."""
+    import torch
+    for seed, mask, dtype in ((21, 0b0001, "f32"), (22, 0b1111, "f32"), (23, 0b1011 | VFIRST, "bf16"),
+                              (24, 0b0001 | VFIRST, "f32")):
+        d = _small(H=5, W=6, N=3, channels=2, batch=2, seed=seed, dtype=dtype, orient_mask=mask & 0xF)
+        dy = np.random.default_rng(seed).standard_normal(d["x"].shape)
+        T = {k: torch.tensor(_f64(d[k]), requires_grad=True) for k in ("x", "delta", "B", "C")}
+        TA = torch.tensor(d["A"].astype(np.float64), requires_grad=True)
+        TD = torch.tensor(d["Dskip"].astype(np.float64), requires_grad=True)
+        y = torch_forward(T["x"], T["delta"], TA, T["B"], T["C"], TD, mask)
+        np.testing.assert_allclose(y.detach().numpy(), _fwd(oracle_mod, d, lib, mask=mask),
+                                   rtol=1e-12, atol=1e-12)
+        (y * torch.tensor(dy)).sum().backward()
+        g = _bwd(oracle_mod, d, dy, lib, mask=mask)
+        want = {"dx": T["x"].grad, "ddelta": T["delta"].grad, "dA": TA.grad, "dB": T["B"].grad,
+                "dC": T["C"].grad, "dDskip": TD.grad}
+        maj = _bwd(oracle_mod, d, dy, lib, mask=mask, majorant=True)
+        for name, ref in want.items():
+            np.testing.assert_allclose(g[name], ref.numpy(), rtol=1e-10, atol=1e-12, err_msg=name)
+            assert np.all(maj[name] >= np.abs(g[name]) * (1 - 1e-12)), name
+
+
+def pin_bwd_finite_difference(oracle_mod, lib=None):
+    """Central differences of sum(dy * y) through the forward oracle, at a few entries of
+    every input, against the gradients."""
+    d = _small(H=4, W=5, N=2, channels=2, batch=1, seed=31, orient_mask=0b0110)
+    rng = np.random.default_rng(31)
+    dy = rng.standard_normal(d["x"].shape)
+    g = _bwd(oracle_mod, d, dy, lib)
+    loss = lambda dd: float(np.sum(dy * _fwd(oracle_mod, dd, lib)))
+    for name, gname in (("x", "dx"), ("delta", "ddelta"), ("A", "dA"), ("B", "dB"), ("C", "dC"),
+                        ("Dskip", "dDskip")):
+        for _ in range(3):
+            idx = tuple(int(rng.integers(0, n)) for n in d[name].shape)
+            plus, minus = dict(d), dict(d)
+            plus[name], minus[name] = d[name].copy(), d[name].copy()
+            v = float(d[name][idx])
+            eps = 1e-2 * max(abs(v), 0.1)
+            plus[name][idx] = np.float32(v + eps)
+            minus[name][idx] = np.float32(v - eps)
+            step = float(plus[name][idx]) - float(minus[name][idx])
+            fd = (loss(plus) - loss(minus)) / step
+            assert abs(fd - g[gname][idx]) <= 2e-4 * (1 + abs(fd)), (name, idx, fd, g[gname][idx])
+
+
 PINS = [pin_closed_form, pin_linsolve, pin_manhattan_constant, pin_golden_3x3,
         pin_1d_reduction, pin_linearity_and_special, pin_orientations, pin_vfirst_closed_form,
-        pin_vfirst_transpose, pin_points_and_maps]
+        pin_vfirst_transpose, pin_points_and_maps, pin_bwd_autograd, pin_bwd_finite_difference]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -356,6 +449,17 @@ MUTATIONS = {
     "vfirst_ignored": ("const int vfirst = p->vfirst;", "const int vfirst = 0;"),
     "vfirst_vertical_without_decay": ("hcol[jj] = abar * hcol[jj] + (dl * Bv) * xv;",
                                       "hcol[jj] = hcol[jj] + (dl * Bv) * xv;"),
+    "bwd_drop_first_scan_term": ("const double dabar = g2[t] * s2_prev + g1[t] * s1_prev;",
+                                 "const double dabar = g2[t] * s2_prev;"),
+    "bwd_adjoint_unshifted_decay": ("g2[t] = Cv * gy + (has_d ? a[AT(ii + 1, jj)] * g2[AT(ii + 1, jj)] : 0.0);",
+                                    "g2[t] = Cv * gy + (has_d ? a[t] * g2[AT(ii + 1, jj)] : 0.0);"),
+    "bwd_dB_without_delta": ("dB[bc + pos] += g1[t] * dl * xv;", "dB[bc + pos] += g1[t] * xv;"),
+    "bwd_ddelta_sign": ("ddelta[map + pos] += dabar * a[t] * Af + g1[t] * Bv * xv;",
+                        "ddelta[map + pos] += -dabar * a[t] * Af + g1[t] * Bv * xv;"),
+    "bwd_dC_first_state": ("dC[bc + pos] += gy * s2[t];", "dC[bc + pos] += gy * s1[t];"),
+    "bwd_skip_missing": ("dx[map + pos] += Dd * gy;", "(void)Dd;"),
+    "bwd_vfirst_adjoint_order": ("g1[t] = g2[t] + (has_d ? a[AT(ii + 1, jj)] * g1[AT(ii + 1, jj)] : 0.0);",
+                                 "g1[t] = g2[t] + (has_r ? a[AT(ii, jj + 1)] * g1[AT(ii, jj + 1)] : 0.0);"),
 }
 
 
