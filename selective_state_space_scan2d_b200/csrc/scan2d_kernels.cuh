@@ -27,9 +27,10 @@
 //     full/empty mbarriers.  The blocks of one chain form a thread-block cluster and the
 //     last warp of a block writes straight into the next block's ring (distributed shared
 //     memory, remote mbarrier arrive), so no compute warp ever waits on a global-memory
-//     fence.  Chains longer than a cluster fall back to a ring in global memory with
-//     release/acquire flags (blocks take their place from a ticket counter, so a block only
-//     waits on blocks that started before it).  Every wait is bounded in time.
+//     fence.  Chains longer than a cluster fall back to a ring in global memory whose
+//     8-byte words carry a row tag beside each value (relaxed loads and stores, no flags or
+//     fences; blocks take their place from a ticket counter, so a block only waits on
+//     blocks that started before it).  Every wait is bounded in time.
 //   * Each warp stages the row tiles of its strip (x, delta for its channels, B, C for all
 //     states) into a private shared-memory ring, by TMA (cp.async.bulk.tensor, mbarrier
 //     completion) when the strides allow, else by plain loads prefetched one row ahead.
