@@ -1,5 +1,6 @@
 /*
- * scan2d.h -- C ABI of the B200 (sm_100a) 2D selective-scan forward (2DMamba).
+ * scan2d.h -- C ABI of the B200 (sm_100a) 2D selective-scan forward (2DMamba) and its
+ * gradients.
  *
  * Operation (sources are web pages on 2DMamba, arXiv 2412.00678):
  *   "2DMamba 精读：从小白到博士" (juejin.cn), section 四.5 "2DMamba 如何扩展到二维？":
@@ -74,6 +75,7 @@ extern "C" {
 
 /* ---- limits ---------------------------------------------------------------------- */
 #define SCAN2D_MAX_N    64     /* states per channel                                   */
+#define SCAN2D_BWD_MAX_N 16    /* states per channel of scan2d_bwd                     */
 #define SCAN2D_NOALLOC_SCRATCH_BYTES 33554432  /* fixed scratch of scan2d_fwd_noalloc (32 MiB) */
 
 /* ---- error codes ----------------------------------------------------------------- */
@@ -90,6 +92,8 @@ extern "C" {
 #define SCAN2D_E_STAGING -10   /* scan2d_fwd_host: staging buffer too small             */
 #define SCAN2D_E_SCRATCH -11   /* scan2d_fwd_noalloc: shape needs more scratch than the
                                   fixed SCAN2D_NOALLOC_SCRATCH_BYTES                    */
+#define SCAN2D_E_WORKSPACE -12 /* scan2d_bwd: workspace smaller than
+                                  scan2d_bwd_workspace_bytes(...)                       */
 
 /*
  * scan2d_fwd -- the 2D selective-scan forward on device buffers.
@@ -171,6 +175,41 @@ int scan2d_fwd_host(const void *x, const void *delta, const float *A, const void
                     const void *C, const float *Dskip, void *y, void *staging,
                     size_t staging_bytes, int batch, int channels, int H, int W, int N,
                     unsigned flags, void *stream);
+
+/*
+ * scan2d_bwd -- gradients of the 2D selective scan (training).  The pages give the forward
+ * only ("2DMamba 精读", section 四.5); these are the chain-rule adjoints of its two recurrences.
+ * For a cotangent dy of y = scan2d_fwd(x, delta, A, B, C, Dskip) they are the derivatives of
+ * L = sum(dy * y):
+ *     gh[p]  = C[p]*dy[p] + Abar[p+e2]*gh[p+e2]     (the vertical scan, backwards)
+ *     ghh[p] = gh[p] + Abar[p+e1]*ghh[p+e1]         (the horizontal scan, backwards)
+ *     dL/dAbar[p] = gh[p]*h[p-e2] + ghh[p]*hh[p-e1]
+ *   dx     = sum_k sum_n ghh*delta*B + Dskip*dy     dB[b,k,n] = sum_d ghh*delta*x
+ *   ddelta = sum_k sum_n (dL/dAbar*Abar*A + ghh*B*x) dC[b,k,n] = sum_d dy*h
+ *   dA[d,n] = sum_{b,k,i,j} dL/dAbar*Abar*delta     dDskip[d] = sum_{b,i,j} dy*x
+ * where e1 / e2 step one column / one row in the orientation's scan direction.
+ *   x, delta, A, B, C, Dskip, flags, shapes : as for scan2d_fwd (Dskip may be NULL, then 0);
+ *   dy, dx, ddelta : device, (batch, channels, H, W), element type of y (fp32; bf16 with
+ *                    SCAN2D_BF16 unless SCAN2D_OUT_F32);
+ *   dA (channels, N), dB and dC (batch, K, N, H, W), dDskip (channels): device fp32; all
+ *                    are overwritten; dDskip may be NULL (not computed);
+ *   workspace      : device buffer of at least scan2d_bwd_workspace_bytes(...) bytes,
+ *                    256-byte aligned, owned by the caller; its contents on entry do not
+ *                    matter and are left undefined.  It holds the forward's vertical state of
+ *                    one orientation (N floats per element) and the strip carries.
+ * Limits: 1 <= N <= SCAN2D_BWD_MAX_N; the default (horizontal-first) scan order only
+ * (SCAN2D_VFIRST returns SCAN2D_E_FLAGS).  Asynchronous on `stream`; outputs must not alias
+ * inputs or each other.  dA, dB, dC and dDskip are sums built with atomic additions, so their
+ * last bits may vary between calls.
+ * Returns 0, or SCAN2D_E_NULL / _DIMS / _N / _FLAGS / _ALIGN / _WORKSPACE / _LAUNCH / _DEVICE.
+ */
+int scan2d_bwd(const void *x, const void *delta, const float *A, const void *B, const void *C,
+               const float *Dskip, const void *dy, void *dx, void *ddelta, float *dA,
+               float *dB, float *dC, float *dDskip, void *workspace, size_t workspace_bytes,
+               int batch, int channels, int H, int W, int N, unsigned flags, void *stream);
+
+/* scan2d_bwd_workspace_bytes -- workspace scan2d_bwd needs for this shape; 0 on bad arguments. */
+size_t scan2d_bwd_workspace_bytes(int batch, int channels, int H, int W, int N, unsigned flags);
 
 /*
  * scan2d_get_device_error -- synchronises `stream`, then returns and clears the first

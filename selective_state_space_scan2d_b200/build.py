@@ -12,9 +12,15 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libscan2d_b200.so")
-SOURCES = [os.path.join(HERE, "csrc", "scan2d.cu")]
-DEPS = SOURCES + [os.path.join(HERE, "csrc", "scan2d_kernels.cuh"),
-                  os.path.join(ROOT, "include", "scan2d.h")]
+OBJDIR = os.path.join(HERE, "_build")
+HEADER = os.path.join(ROOT, "include", "scan2d.h")
+# each translation unit with the files it includes; they compile in parallel
+UNITS = {
+    os.path.join(HERE, "csrc", "scan2d.cu"): [os.path.join(HERE, "csrc", "scan2d_kernels.cuh"), HEADER],
+    os.path.join(HERE, "csrc", "scan2d_bwd.cu"): [HEADER],
+}
+SOURCES = list(UNITS)
+DEPS = SOURCES + sorted({d for deps in UNITS.values() for d in deps})
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -25,21 +31,46 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
+def _obj(src: str) -> str:
+    return os.path.join(OBJDIR, os.path.splitext(os.path.basename(src))[0] + ".o")
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and os.path.exists(LIB):
         t = os.path.getmtime(LIB)
         if all(os.path.getmtime(d) <= t for d in DEPS):
             return LIB
+    os.makedirs(OBJDIR, exist_ok=True)
+    flags = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2"]
+    if verbose:
+        flags.insert(0, "-Xptxas=-v")
+    procs = []
+    for src, deps in UNITS.items():
+        obj = _obj(src)
+        fresh = (not force and os.path.exists(obj) and
+                 all(os.path.getmtime(d) <= os.path.getmtime(obj) for d in [src, *deps]))
+        if fresh:
+            continue
+        tmp = obj + f".tmp{os.getpid()}"
+        procs.append((obj, tmp, subprocess.Popen([nvcc(), *flags, "-c", "-o", tmp, src],
+                                                 stdout=subprocess.PIPE, stderr=subprocess.STDOUT,
+                                                 text=True)))
+    failed = []
+    for obj, tmp, proc in procs:
+        out, _ = proc.communicate()
+        if proc.returncode != 0:
+            failed.append(out)
+        else:
+            if verbose:
+                sys.stderr.write(out)
+            os.replace(tmp, obj)
+    if failed:
+        raise RuntimeError("nvcc failed:\n" + "\n".join(failed))
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2",
-           "-shared", "-o", tmp, *SOURCES]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    res = subprocess.run(cmd, capture_output=True, text=True)
+    res = subprocess.run([nvcc(), *ARCH, "-shared", "-o", tmp, *(_obj(s) for s in SOURCES)],
+                         capture_output=True, text=True)
     if res.returncode != 0:
-        raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
-    if verbose:
-        sys.stderr.write(res.stdout + res.stderr)
+        raise RuntimeError("nvcc link failed:\n" + res.stdout + res.stderr)
     os.replace(tmp, LIB)
     return LIB
 

@@ -728,6 +728,7 @@ const char* scan2d_strerror(int code) {
     case SCAN2D_E_DEVICE: return "no usable sm_100 CUDA device";
     case SCAN2D_E_STAGING: return "staging buffer too small";
     case SCAN2D_E_SCRATCH: return "scan2d_fwd_noalloc: the shape needs more scratch than SCAN2D_NOALLOC_SCRATCH_BYTES";
+    case SCAN2D_E_WORKSPACE: return "scan2d_bwd: workspace smaller than scan2d_bwd_workspace_bytes";
     default: return "unknown error";
   }
 }

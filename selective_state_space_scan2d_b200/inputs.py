@@ -27,7 +27,7 @@ import numpy as np
 
 ORIENT_TL, ORIENT_TR, ORIENT_BL, ORIENT_BR = 1, 2, 4, 8
 
-_TENSOR_ID = {"x": 1, "delta": 2, "B": 3, "C": 4, "Dskip": 5, "pad": 6, "mask": 7, "A": 8}
+_TENSOR_ID = {"x": 1, "delta": 2, "B": 3, "C": 4, "Dskip": 5, "pad": 6, "mask": 7, "A": 8, "dy": 9}
 
 
 @dataclasses.dataclass(frozen=True)
@@ -154,3 +154,12 @@ def make_inputs(w: Workload | str, seed: int = 0) -> dict:
         raise ValueError(w.dtype)
     return dict(x=x, delta=delta, A=np.ascontiguousarray(A, dtype=np.float32), B=B, C=C,
                 Dskip=Dskip, workload=w, orient_mask=w.orient_mask, vfirst=w.vfirst)
+
+
+def make_cotangent(w: Workload | str, seed: int = 0, out_f32: bool = False) -> np.ndarray:
+    """A seeded cotangent dy for the gradients: N(0, 1) values of y's shape, as bf16 bits
+    when y is bf16 (bf16 inputs without fp32 output), else float32."""
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    dy = _rng(seed, "dy").standard_normal((w.batch, w.channels, w.H, w.W), dtype=np.float32)
+    return f32_to_bf16_bits(dy) if (w.dtype == "bf16" and not out_f32) else dy

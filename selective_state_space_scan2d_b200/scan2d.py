@@ -35,6 +35,11 @@ _lib.scan2d_host_staging_bytes.argtypes = [_i, _i, _i, _i, _i, _u]
 _lib.scan2d_host_staging_bytes.restype = _sz
 _lib.scan2d_fwd_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i, _i, _i, _i, _i, _u, _vp]
 _lib.scan2d_fwd_host.restype = _i
+_lib.scan2d_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                            _i, _i, _i, _i, _i, _u, _vp]
+_lib.scan2d_bwd.restype = _i
+_lib.scan2d_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _u]
+_lib.scan2d_bwd_workspace_bytes.restype = _sz
 _lib.scan2d_get_device_error.argtypes = [_vp]
 _lib.scan2d_get_device_error.restype = _i
 _lib.scan2d_strerror.argtypes = [_i]
@@ -51,7 +56,9 @@ SCAN2D_OR_TR = 0x20
 SCAN2D_OR_BL = 0x40
 SCAN2D_OR_BR = 0x80
 SCAN2D_E_SCRATCH = -11
+SCAN2D_E_WORKSPACE = -12
 SCAN2D_NOALLOC_SCRATCH_BYTES = 32 << 20
+SCAN2D_BWD_MAX_N = 16
 
 
 class Scan2dError(RuntimeError):
@@ -171,6 +178,43 @@ def scan2d_fwd_noalloc(x, delta, A, B, C, Dskip, y, flags=None, stream=None):
     if rc:
         raise Scan2dError(rc, "scan2d_fwd_noalloc")
     return y
+
+
+def scan2d_bwd_workspace_bytes(batch, channels, H, W, N, flags) -> int:
+    return int(_lib.scan2d_bwd_workspace_bytes(batch, channels, H, W, N, flags))
+
+
+def scan2d_bwd(x, delta, A, B, C, Dskip, dy, flags=None, workspace=None, stream=None) -> dict:
+    """Gradients of sum(dy * scan2d_fwd(x, delta, A, B, C, Dskip)) on CUDA tensors
+    (asynchronous on `stream`): a dict with dx, ddelta (the layout and element type of y),
+    dA (channels, N), dB and dC (the layout of B), dDskip (channels,), all fp32 but dx and
+    ddelta.  `workspace` (a uint8 CUDA tensor of at least scan2d_bwd_workspace_bytes(...)
+    bytes) is allocated here when not given."""
+    torch = _torch()
+    _check(x, delta, A, B, C, Dskip, "cuda")
+    batch, D, H, W, N, K = _dims(x, B, A)
+    if flags is None:
+        flags = flags_for(x.dtype == torch.bfloat16, (1 << K) - 1)
+    out_dtype = torch.float32 if (x.dtype == torch.float32 or flags & SCAN2D_OUT_F32) else torch.bfloat16
+    if dy.dtype != out_dtype or tuple(dy.shape) != (batch, D, H, W) or not dy.is_contiguous() or not dy.is_cuda:
+        raise ValueError("dy must be a contiguous CUDA tensor of the shape and dtype of y")
+    need = scan2d_bwd_workspace_bytes(batch, D, H, W, N, flags)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    dev = x.device
+    g = {"dx": torch.empty((batch, D, H, W), dtype=out_dtype, device=dev),
+         "ddelta": torch.empty((batch, D, H, W), dtype=out_dtype, device=dev),
+         "dA": torch.empty((D, N), dtype=torch.float32, device=dev),
+         "dB": torch.empty(tuple(B.shape), dtype=torch.float32, device=dev),
+         "dC": torch.empty(tuple(C.shape), dtype=torch.float32, device=dev),
+         "dDskip": torch.empty((D,), dtype=torch.float32, device=dev)}
+    rc = _lib.scan2d_bwd(_ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(Dskip), _ptr(dy),
+                         *(_ptr(g[k]) for k in ("dx", "ddelta", "dA", "dB", "dC", "dDskip")),
+                         _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
+                         batch, D, H, W, N, flags, _stream_handle(stream))
+    if rc:
+        raise Scan2dError(rc, "scan2d_bwd")
+    return g
 
 
 PLAN_FIELDS = ("launches", "grid", "threads", "smem", "nseg", "cols", "wpc", "mode", "ng",

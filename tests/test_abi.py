@@ -117,6 +117,35 @@ def test_staging_size_and_host_checks(lib):
     assert r.scan2d_fwd_host(P, P, P, P, P, None, P, P + 16, n, 1, 4, 8, 8, 4, 0x10, None) == m["SCAN2D_E_ALIGN"]
 
 
+def test_bwd_workspace_size_and_host_checks(lib):
+    m = _header_macros()
+    assert lib.SCAN2D_E_WORKSPACE == m["SCAN2D_E_WORKSPACE"]
+    assert lib.SCAN2D_BWD_MAX_N == m["SCAN2D_BWD_MAX_N"]
+    # hsave: N floats per element (4 * 64 * 4); three strip-carry arrays of H * strips * N
+    # floats per channel (8 * 1 * 4 * 4 channels), each rounded up to 256 bytes
+    n = lib.scan2d_bwd_workspace_bytes(1, 4, 8, 8, 4, 0x10)
+    assert n == 4 * 64 * 4 * 4 + 3 * 512
+    # bf16 y with several orientations adds two fp32 accumulators of the element count
+    nb = lib.scan2d_bwd_workspace_bytes(1, 4, 8, 8, 4, 0x31)
+    assert nb == n + 2 * 4 * 64 * 4
+    assert lib.scan2d_bwd_workspace_bytes(1, 4, 8, 8, 17, 0x10) == 0
+    r = lib.raw()
+    dims = (1, 4, 8, 8, 4)
+    call = lambda *ptrs, size=n, flags=0x10, d=dims: r.scan2d_bwd(*ptrs, size, *d, flags, None)
+    good = [P] * 14
+    good[5] = None                                     # Dskip may be NULL
+    assert call(*good, flags=0x18) == m["SCAN2D_E_FLAGS"]          # vertical-first: forward only
+    assert call(*good, d=(1, 4, 8, 8, 17)) == m["SCAN2D_E_N"]
+    assert call(*good, size=n - 1) == m["SCAN2D_E_WORKSPACE"]
+    for k in (0, 6, 7, 13):
+        bad = list(good)
+        bad[k] = None
+        assert call(*bad) == m["SCAN2D_E_NULL"], k
+    bad = list(good)
+    bad[13] = P + 16                                   # workspace must be 256-byte aligned
+    assert call(*bad) == m["SCAN2D_E_ALIGN"]
+
+
 def test_valid_call_without_a_gpu_fails_loudly(lib):
     """No CPU fallback: with valid arguments and no usable device the call is an error."""
     import torch
