@@ -16,14 +16,15 @@
 // Design.  The adjoint runs against the forward's direction in both dimensions, and needs the
 // forward's vertical state h of the row before each row.  The forward keeps that state in
 // registers and never stores it, so the backward first recomputes it and stores it (N floats
-// per element, one orientation at a time).  No kernel here waits on another warp:
+// per element, one orientation at a time, strip-major: the 8 columns x N states x 8 channels of
+// one warp's row are one contiguous 4 KB block).  No kernel here waits on another warp:
 //   1. k_pre    walks each strip's rows backwards, carrying the adjoint's vertical state in
 //               registers.  For every (row, strip, channel, state) it writes what the strip
 //               adds to the two horizontal carries when it starts from zero (forward: the hh
 //               leaving the strip; adjoint: a*ghh leaving it) and the product of a across the
 //               strip: a carry that enters the strip leaves it multiplied by that product.
-//   2. k_carry  runs the two short recurrences across the strips of every row and replaces
-//               those terms in place by the carry that enters each strip.
+//   2. k_carry  runs the two short recurrences across the strips of every row and writes the
+//               carry that enters each strip.
 //   3. k_states walks each strip's rows forwards from the known carries and stores h.
 //   4. k_main   walks each strip's rows backwards from the known carries, with h of the row
 //               before read back, and produces every gradient.
@@ -62,10 +63,13 @@ struct Args {
   float* dB;
   float* dC;
   float* dDskip;            // may be null
-  float* hsave;             // (batch, channels, N, H, W): forward vertical state of one orientation
-  float* cf;                // (batch, channels, H, S, N): forward horizontal carry terms
-  float* cb;                //   adjoint horizontal carry terms
+  float* hsave;             // (batch, H, S, channels, N, 8): forward vertical state of one
+                            // orientation, strip-major so that a warp's row is contiguous
+  float* tf;                // (batch, H, S, channels, N): forward horizontal carry terms
+  float* tb;                //   adjoint horizontal carry terms
   float* beta;              //   product of a across the strip
+  float* cf;                //   forward carry entering the strip
+  float* cb;                //   adjoint carry entering the strip
   long long tasks;          // warps: batch * S * channel groups
   int batch, channels, H, W, N, K, S, ncg;
   int k;                    // orientation index: B_k, C_k, dB_k, dC_k
@@ -73,7 +77,6 @@ struct Args {
   int first, last;          // first / last orientation of the call
   int vec_in;               // input rows allow 16-byte loads
   int vec_g;                // dy rows allow 16-byte loads
-  int vec_h;                // hsave rows allow 16-byte access (W % 4 == 0)
   int vec2;                 // W even and outputs aligned: 2-column stores and atomics
 };
 
@@ -86,54 +89,6 @@ __device__ __forceinline__ float ex2_approx(float v) {
 __device__ __forceinline__ float to_f(float v) { return v; }
 __device__ __forceinline__ float to_f(uint16_t v) { return __uint_as_float(static_cast<uint32_t>(v) << 16); }
 
-// 8 consecutive values of a row starting at column j0; columns at or beyond W read as 0.
-template <typename T>
-__device__ __forceinline__ void load8(const T* row, int j0, int W, bool vec, float (&v)[kCols]) {
-  if (vec && j0 + kCols <= W) {
-    if constexpr (sizeof(T) == 4) {
-      const float4 a = __ldg(reinterpret_cast<const float4*>(row + j0));
-      const float4 b = __ldg(reinterpret_cast<const float4*>(row + j0 + 4));
-      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-      v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-    } else {
-      const uint4 a = __ldg(reinterpret_cast<const uint4*>(row + j0));
-      const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        v[2 * e] = __uint_as_float(w[e] << 16);
-        v[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
-      }
-    }
-  } else {
-#pragma unroll
-    for (int c = 0; c < kCols; ++c) v[c] = (j0 + c < W) ? to_f(row[j0 + c]) : 0.f;
-  }
-}
-
-// Plain (coherent) loads for buffers written by an earlier kernel of the same call.
-__device__ __forceinline__ void load8_ws(const float* row, int j0, int W, bool vec, float (&v)[kCols]) {
-  if (vec && j0 + kCols <= W) {
-    const float4 a = *reinterpret_cast<const float4*>(row + j0);
-    const float4 b = *reinterpret_cast<const float4*>(row + j0 + 4);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-  } else {
-#pragma unroll
-    for (int c = 0; c < kCols; ++c) v[c] = (j0 + c < W) ? row[j0 + c] : 0.f;
-  }
-}
-
-__device__ __forceinline__ void store8_ws(float* row, int j0, int W, bool vec, const float (&v)[kCols]) {
-  if (vec && j0 + kCols <= W) {
-    *reinterpret_cast<float4*>(row + j0) = make_float4(v[0], v[1], v[2], v[3]);
-    *reinterpret_cast<float4*>(row + j0 + 4) = make_float4(v[4], v[5], v[6], v[7]);
-  } else {
-#pragma unroll
-    for (int c = 0; c < kCols; ++c)
-      if (j0 + c < W) row[j0 + c] = v[c];
-  }
-}
-
 // One of the lane's 8 columns, chosen by two lane bits (keeps the register arrays static).
 __device__ __forceinline__ float pick(const float (&v)[kCols], bool m2, bool m1, int e) {
   const float lo = m1 ? v[2 + e] : v[e];
@@ -142,7 +97,7 @@ __device__ __forceinline__ float pick(const float (&v)[kCols], bool m2, bool m1,
 }
 
 struct Task {
-  int b, s, d, q, j0;
+  int b, s, cgi, d, q, j0;
   bool act;
 };
 
@@ -150,11 +105,11 @@ __device__ __forceinline__ bool decode(const Args& p, Task& t) {
   const long long task = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
   if (task >= p.tasks) return false;
   const int lane = threadIdx.x & 31;
-  const int cgi = static_cast<int>(task % p.ncg);
+  t.cgi = static_cast<int>(task % p.ncg);
   const long long rest = task / p.ncg;
   t.s = static_cast<int>(rest % p.S);
   t.b = static_cast<int>(rest / p.S);
-  t.d = cgi * kCh + (lane >> 2);
+  t.d = t.cgi * kCh + (lane >> 2);
   t.q = lane & 3;
   t.j0 = t.s * kCols;
   t.act = t.d < p.channels;
@@ -164,33 +119,138 @@ __device__ __forceinline__ bool decode(const Args& p, Task& t) {
 // scan-order row ii of this orientation -> stored row
 __device__ __forceinline__ int row_of(const Args& p, int ii) { return p.flipH ? p.H - 1 - ii : ii; }
 
-// index of (b, d, row i, strip s, state n) in the strip-carry arrays
+// index of (b, row i, strip s, channel d, state n) in the strip-carry arrays; channels are
+// padded to whole groups of 8, so a warp's 8 x N values start on a 32-byte boundary
 __device__ __forceinline__ size_t carry_idx(const Args& p, int b, int d, int i, int s, int n) {
-  return ((((size_t)b * p.channels + d) * p.H + i) * p.S + s) * p.N + n;
+  return ((((size_t)b * p.H + i) * p.S + s) * (size_t)(p.ncg * kCh) + d) * p.N + n;
+}
+
+// first float of the 8 columns of (b, row i, strip s, channel d, state n) in hsave
+__device__ __forceinline__ size_t hs_idx(const Args& p, int b, int d, int i, int s, int n) {
+  return carry_idx(p, b, d, i, s, n) * kCols;
+}
+
+__device__ __forceinline__ void st8(float* dst, const float (&v)[kCols]) {
+  *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+  *reinterpret_cast<float4*>(dst + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+__device__ __forceinline__ void lds8(const float* src, float (&v)[kCols]) {
+  const float4 a = *reinterpret_cast<const float4*>(src);
+  const float4 b = *reinterpret_cast<const float4*>(src + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// ---- per-warp row staging -------------------------------------------------------------------------
+// Each warp stages the rows it walks into two shared-memory buffers, one row ahead:
+//   * the inputs (x, delta, dy of its 8 channels, B and C of all states, 8 columns each) are
+//     loaded into registers while the current row is computed and stored to shared memory
+//     (as fp32) after it, element by element, so any alignment works;
+//   * the workspace blocks (strip carries, saved states: contiguous and 32-byte aligned by
+//     construction) are copied with cp.async.
+// Buffer layout, in floats:
+constexpr int kOffX = 0;                                  // [8 channels][8 columns]
+constexpr int kOffD = kOffX + kCh * kCols;                // delta
+constexpr int kOffB = kOffD + kCh * kCols;                // [N states][8 columns]
+constexpr int kOffC = kOffB + kMaxNBwd * kCols;
+constexpr int kOffG = kOffC + kMaxNBwd * kCols;           // dy [8 channels][8 columns]
+constexpr int kOffCF = kOffG + kCh * kCols;               // forward carries [8 channels * N]
+constexpr int kOffCB = kOffCF + kCh * kMaxNBwd;           // adjoint carries
+constexpr int kOffH = kOffCB + kCh * kMaxNBwd;            // saved states [8 channels * N][8 columns]
+constexpr int kBufPre = kOffCF;                           // floats per buffer: k_pre
+constexpr int kBufStates = kOffCB;                        //   k_states
+constexpr int kBufMain = kOffH + kCh * kMaxNBwd * kCols;  //   k_main
+
+template <typename Tin, typename Tg, int NG, bool WITH_C, bool WITH_G>
+struct InputPrefetch {
+  Tin x[2], dl[2];
+  Tg gy[2];
+  Tin bv[NG], cv[NG];
+  size_t xo[2], bo[NG];        // element offsets without the row term
+  bool xok[2], bok[NG];
+
+  __device__ __forceinline__ void init(const Args& p, const Task& t, int lane) {
+    const size_t HW = (size_t)p.H * p.W;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int e = lane + 32 * k, ch = e >> 3, col = e & 7;
+      const int d = t.cgi * kCh + ch, j = t.j0 + col;
+      xok[k] = d < p.channels && j < p.W;
+      xo[k] = xok[k] ? ((size_t)t.b * p.channels + d) * HW + j : 0;
+    }
+#pragma unroll
+    for (int k = 0; k < NG; ++k) {
+      const int e = lane + 32 * k, n = e >> 3, col = e & 7;
+      const int j = t.j0 + col;
+      bok[k] = n < p.N && j < p.W;
+      bo[k] = bok[k] ? (((size_t)t.b * p.K + p.k) * p.N + n) * HW + j : 0;
+    }
+  }
+  __device__ __forceinline__ void load(const Args& p, int i) {
+    const size_t r = (size_t)i * p.W;
+    const Tin* X = static_cast<const Tin*>(p.x);
+    const Tin* Dl = static_cast<const Tin*>(p.delta);
+    const Tg* G = static_cast<const Tg*>(p.dy);
+    const Tin* Bm = static_cast<const Tin*>(p.B);
+    const Tin* Cm = static_cast<const Tin*>(p.C);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      x[k] = xok[k] ? __ldg(X + xo[k] + r) : Tin(0);
+      dl[k] = xok[k] ? __ldg(Dl + xo[k] + r) : Tin(0);
+      if (WITH_G) gy[k] = xok[k] ? __ldg(G + xo[k] + r) : Tg(0);
+    }
+#pragma unroll
+    for (int k = 0; k < NG; ++k) {
+      bv[k] = bok[k] ? __ldg(Bm + bo[k] + r) : Tin(0);
+      if (WITH_C) cv[k] = bok[k] ? __ldg(Cm + bo[k] + r) : Tin(0);
+    }
+  }
+  __device__ __forceinline__ void store(float* buf, int lane) const {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      buf[kOffX + lane + 32 * k] = to_f(x[k]);
+      buf[kOffD + lane + 32 * k] = to_f(dl[k]);
+      if (WITH_G) buf[kOffG + lane + 32 * k] = to_f(gy[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < NG; ++k) {
+      buf[kOffB + lane + 32 * k] = to_f(bv[k]);
+      if (WITH_C) buf[kOffC + lane + 32 * k] = to_f(cv[k]);
+    }
+  }
+};
+
+// cp.async of n16 16-byte chunks from src to dst, spread over the warp's lanes
+__device__ __forceinline__ void copy_block(float* dst, const float* src, int n16, int lane) {
+  for (int c = lane; c < n16; c += 32) cp_async16(dst + 4 * c, src + 4 * c);
 }
 
 // ---- 1. strip terms of the two horizontal carries ---------------------------------------------
 template <typename Tin, typename Tg, int NG, bool FW>
 __global__ void __launch_bounds__(kWarps * 32) k_pre(const Args p) {
+  extern __shared__ __align__(16) float smem[];
   Task t;
   if (!decode(p, t)) return;
-  const size_t HW = (size_t)p.H * p.W;
-  const size_t map = ((size_t)t.b * p.channels + (t.act ? t.d : 0)) * HW;
-  const Tin* xm = static_cast<const Tin*>(p.x) + map;
-  const Tin* dm = static_cast<const Tin*>(p.delta) + map;
-  const Tg* gm = static_cast<const Tg*>(p.dy) + map;
+  const int lane = threadIdx.x & 31, cg = lane >> 2;
+  float* buf0 = smem + (threadIdx.x >> 5) * 2 * kBufPre;
   float A2[NG];
   bool nok[NG];
-  const Tin* Bp[NG];
-  const Tin* Cp[NG];
 #pragma unroll
   for (int g = 0; g < NG; ++g) {
     const int n = t.q + 4 * g;
     nok[g] = n < p.N;
     A2[g] = (t.act && nok[g]) ? p.A[(size_t)t.d * p.N + n] * kLog2e : 0.f;
-    const size_t plane = (((size_t)t.b * p.K + p.k) * p.N + (nok[g] ? n : 0)) * HW;
-    Bp[g] = static_cast<const Tin*>(p.B) + plane;
-    Cp[g] = static_cast<const Tin*>(p.C) + plane;
   }
   float V[NG][kCols];                      // a*gh of the row after (in forward order)
 #pragma unroll
@@ -198,27 +258,25 @@ __global__ void __launch_bounds__(kWarps * 32) k_pre(const Args p) {
 #pragma unroll
     for (int c = 0; c < kCols; ++c) V[g][c] = 0.f;
 
-  for (int ii = p.H - 1; ii >= 0; --ii) {
+  InputPrefetch<Tin, Tg, NG, true, true> pf;
+  pf.init(p, t, lane);
+  pf.load(p, row_of(p, p.H - 1));
+  pf.store(buf0, lane);
+  __syncwarp();
+  for (int e = 0; e < p.H; ++e) {
+    const int ii = p.H - 1 - e;
     const int i = row_of(p, ii);
+    float* cur = buf0 + (e & 1) * kBufPre;
+    if (ii > 0) pf.load(p, row_of(p, ii - 1));
     float xv[kCols], dl[kCols], gy[kCols];
-    if (t.act) {
-      load8(xm + (size_t)i * p.W, t.j0, p.W, p.vec_in, xv);
-      load8(dm + (size_t)i * p.W, t.j0, p.W, p.vec_in, dl);
-      load8(gm + (size_t)i * p.W, t.j0, p.W, p.vec_g, gy);
-    } else {
-#pragma unroll
-      for (int c = 0; c < kCols; ++c) xv[c] = dl[c] = gy[c] = 0.f;
-    }
+    lds8(cur + kOffX + cg * kCols, xv);
+    lds8(cur + kOffD + cg * kCols, dl);
+    lds8(cur + kOffG + cg * kCols, gy);
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
       float bv[kCols], cv[kCols];
-      if (nok[g]) {
-        load8(Bp[g] + (size_t)i * p.W, t.j0, p.W, p.vec_in, bv);
-        load8(Cp[g] + (size_t)i * p.W, t.j0, p.W, p.vec_in, cv);
-      } else {
-#pragma unroll
-        for (int c = 0; c < kCols; ++c) bv[c] = cv[c] = 0.f;
-      }
+      lds8(cur + kOffB + (t.q + 4 * g) * kCols, bv);
+      lds8(cur + kOffC + (t.q + 4 * g) * kCols, cv);
       float a[kCols];
       float prod = 1.f;
 #pragma unroll
@@ -228,103 +286,133 @@ __global__ void __launch_bounds__(kWarps * 32) k_pre(const Args p) {
       }
       float r = 0.f;                        // forward: hh leaving the strip, from zero
 #pragma unroll
-      for (int e = 0; e < kCols; ++e) {
-        const int c = FW ? kCols - 1 - e : e;
+      for (int k = 0; k < kCols; ++k) {
+        const int c = FW ? kCols - 1 - k : k;
         r = fmaf(a[c], r, (dl[c] * xv[c]) * bv[c]);
       }
       float hc = 0.f;                       // adjoint: a*ghh leaving the strip, from zero
 #pragma unroll
-      for (int e = 0; e < kCols; ++e) {
-        const int c = FW ? e : kCols - 1 - e;
+      for (int k = 0; k < kCols; ++k) {
+        const int c = FW ? k : kCols - 1 - k;
         const float gh = fmaf(cv[c], gy[c], V[g][c]);
         V[g][c] = a[c] * gh;
         hc = a[c] * (gh + hc);
       }
       if (t.act && nok[g]) {
         const size_t ci = carry_idx(p, t.b, t.d, i, t.s, t.q + 4 * g);
-        p.cf[ci] = r;
-        p.cb[ci] = hc;
+        p.tf[ci] = r;
+        p.tb[ci] = hc;
         p.beta[ci] = prod;
       }
     }
+    if (ii > 0) pf.store(buf0 + ((e + 1) & 1) * kBufPre, lane);
+    __syncwarp();
   }
 }
 
 // ---- 2. carries entering each strip -----------------------------------------------------------
-// One thread per (b, d, row, state): forward carries in the forward strip order, adjoint
-// carries in the reverse order; each term is replaced by the carry that enters its strip.
+// One thread per (b, row, channel, state): the forward carries in the forward strip order and
+// the adjoint carries in the reverse order.  Adjacent threads hold adjacent (channel, state),
+// so every strip step is one coalesced access per warp; the terms of kChunk strips are loaded
+// before any of them is used, so those loads are in flight together.
+constexpr int kChunk = 8;
+
 __global__ void __launch_bounds__(256) k_carry(const Args p, int fw) {
-  const long long total = (long long)p.batch * p.channels * p.H * p.N;
+  const long long dn = (long long)p.ncg * kCh * p.N;
+  const long long total = (long long)p.batch * p.H * dn;
   const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t >= total) return;
-  const int n = static_cast<int>(t % p.N);
-  const size_t base = (size_t)(t / p.N) * p.S * p.N + n;
-  float carry = 0.f;
-  for (int e = 0; e < p.S; ++e) {
-    const int s = fw ? p.S - 1 - e : e;
-    const size_t ci = base + (size_t)s * p.N;
-    const float term = p.cf[ci];
-    p.cf[ci] = carry;
-    carry = fmaf(p.beta[ci], carry, term);
-  }
-  carry = 0.f;
-  for (int e = 0; e < p.S; ++e) {
-    const int s = fw ? e : p.S - 1 - e;
-    const size_t ci = base + (size_t)s * p.N;
-    const float term = p.cb[ci];
-    p.cb[ci] = carry;
-    carry = fmaf(p.beta[ci], carry, term);
+  if ((t % dn) / p.N >= p.channels) return;        // padding channel
+  const size_t base = (size_t)(t / dn) * p.S * dn + (size_t)(t % dn);
+  const float* __restrict__ tf = p.tf;
+  const float* __restrict__ tb = p.tb;
+  const float* __restrict__ be = p.beta;
+  float* __restrict__ cf = p.cf;
+  float* __restrict__ cb = p.cb;
+  for (int dir = 0; dir < 2; ++dir) {
+    const bool rev = (dir == 0) == (fw != 0);      // strips walked from the last one
+    const float* __restrict__ term = dir == 0 ? tf : tb;
+    float* __restrict__ out = dir == 0 ? cf : cb;
+    float carry = 0.f;
+    for (int e0 = 0; e0 < p.S; e0 += kChunk) {
+      float tv[kChunk], bv[kChunk];
+#pragma unroll
+      for (int e = 0; e < kChunk; ++e) {
+        const int s = rev ? p.S - 1 - (e0 + e) : e0 + e;
+        const bool ok = e0 + e < p.S;
+        tv[e] = ok ? __ldg(term + base + (size_t)s * dn) : 0.f;
+        bv[e] = ok ? __ldg(be + base + (size_t)s * dn) : 1.f;
+      }
+#pragma unroll
+      for (int e = 0; e < kChunk; ++e) {
+        const int s = rev ? p.S - 1 - (e0 + e) : e0 + e;
+        if (e0 + e < p.S) out[base + (size_t)s * dn] = carry;
+        carry = fmaf(bv[e], carry, tv[e]);
+      }
+    }
   }
 }
 
 // ---- 3. forward vertical state of every element -----------------------------------------------
 template <typename Tin, int NG, bool FW>
 __global__ void __launch_bounds__(kWarps * 32) k_states(const Args p) {
+  extern __shared__ __align__(16) float smem[];
   Task t;
   if (!decode(p, t)) return;
-  if (!t.act) return;                       // no shuffles in this kernel
-  const size_t HW = (size_t)p.H * p.W;
-  const size_t map = ((size_t)t.b * p.channels + t.d) * HW;
-  const Tin* xm = static_cast<const Tin*>(p.x) + map;
-  const Tin* dm = static_cast<const Tin*>(p.delta) + map;
+  const int lane = threadIdx.x & 31, cg = lane >> 2;
+  float* buf0 = smem + (threadIdx.x >> 5) * 2 * kBufStates;
   float A2[NG];
   bool nok[NG];
-  const Tin* Bp[NG];
-  float* hs[NG];
 #pragma unroll
   for (int g = 0; g < NG; ++g) {
     const int n = t.q + 4 * g;
     nok[g] = n < p.N;
-    A2[g] = nok[g] ? p.A[(size_t)t.d * p.N + n] * kLog2e : 0.f;
-    Bp[g] = static_cast<const Tin*>(p.B) + (((size_t)t.b * p.K + p.k) * p.N + (nok[g] ? n : 0)) * HW;
-    hs[g] = p.hsave + (((size_t)t.b * p.channels + t.d) * p.N + (nok[g] ? n : 0)) * HW;
+    A2[g] = (t.act && nok[g]) ? p.A[(size_t)t.d * p.N + n] * kLog2e : 0.f;
   }
   float h[NG][kCols];
 #pragma unroll
   for (int g = 0; g < NG; ++g)
 #pragma unroll
     for (int c = 0; c < kCols; ++c) h[g][c] = 0.f;
+  const int n16 = 2 * p.N;                 // 8 channels x N carries, in 16-byte chunks
 
+  InputPrefetch<Tin, float, NG, false, false> pf;
+  pf.init(p, t, lane);
+  pf.load(p, row_of(p, 0));
+  copy_block(buf0 + kOffCF, p.cf + carry_idx(p, t.b, t.cgi * kCh, row_of(p, 0), t.s, 0), n16, lane);
+  cp_commit();
+  pf.store(buf0, lane);
   for (int ii = 0; ii < p.H; ++ii) {
     const int i = row_of(p, ii);
+    float* cur = buf0 + (ii & 1) * kBufStates;
+    float* nxt = buf0 + ((ii + 1) & 1) * kBufStates;
+    if (ii + 1 < p.H) {
+      pf.load(p, row_of(p, ii + 1));
+      copy_block(nxt + kOffCF, p.cf + carry_idx(p, t.b, t.cgi * kCh, row_of(p, ii + 1), t.s, 0), n16, lane);
+    }
+    cp_commit();
+    cp_wait1();
+    __syncwarp();
     float xv[kCols], dl[kCols];
-    load8(xm + (size_t)i * p.W, t.j0, p.W, p.vec_in, xv);
-    load8(dm + (size_t)i * p.W, t.j0, p.W, p.vec_in, dl);
+    lds8(cur + kOffX + cg * kCols, xv);
+    lds8(cur + kOffD + cg * kCols, dl);
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
-      if (!nok[g]) continue;
+      const int n = t.q + 4 * g;
       float bv[kCols];
-      load8(Bp[g] + (size_t)i * p.W, t.j0, p.W, p.vec_in, bv);
-      float r = p.cf[carry_idx(p, t.b, t.d, i, t.s, t.q + 4 * g)];
+      lds8(cur + kOffB + n * kCols, bv);
+      float r = nok[g] ? cur[kOffCF + cg * p.N + n] : 0.f;
 #pragma unroll
-      for (int e = 0; e < kCols; ++e) {
-        const int c = FW ? kCols - 1 - e : e;
+      for (int k = 0; k < kCols; ++k) {
+        const int c = FW ? kCols - 1 - k : k;
         const float a = ex2_approx(dl[c] * A2[g]);
         r = fmaf(a, r, (dl[c] * xv[c]) * bv[c]);
         h[g][c] = fmaf(a, h[g][c], r);
       }
-      store8_ws(hs[g] + (size_t)i * p.W, t.j0, p.W, p.vec_h, h[g]);
+      if (t.act && nok[g]) st8(p.hsave + hs_idx(p, t.b, t.d, i, t.s, n), h[g]);
     }
+    if (ii + 1 < p.H) pf.store(nxt, lane);
+    __syncwarp();
   }
 }
 
@@ -353,30 +441,22 @@ __device__ __forceinline__ void put2(Tg* out, size_t idx, float v0, float v1, bo
 
 template <typename Tin, typename Tg, int NG, bool FW>
 __global__ void __launch_bounds__(kWarps * 32) k_main(const Args p) {
+  extern __shared__ __align__(16) float smem[];
   Task t;
   if (!decode(p, t)) return;
-  const int lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31, cg = lane >> 2;
   const bool hi = lane & 16, m8 = lane & 8, m4 = lane & 4, m2 = lane & 2, m1 = lane & 1;
+  float* buf0 = smem + (threadIdx.x >> 5) * 2 * kBufMain;
   const size_t HW = (size_t)p.H * p.W;
   const size_t map = ((size_t)t.b * p.channels + (t.act ? t.d : 0)) * HW;
-  const Tin* xm = static_cast<const Tin*>(p.x) + map;
-  const Tin* dm = static_cast<const Tin*>(p.delta) + map;
-  const Tg* gm = static_cast<const Tg*>(p.dy) + map;
   float A2[NG], Af[NG];
   bool nok[NG];
-  const Tin* Bp[NG];
-  const Tin* Cp[NG];
-  const float* hs[NG];
 #pragma unroll
   for (int g = 0; g < NG; ++g) {
     const int n = t.q + 4 * g;
     nok[g] = n < p.N;
     Af[g] = (t.act && nok[g]) ? p.A[(size_t)t.d * p.N + n] : 0.f;
     A2[g] = Af[g] * kLog2e;
-    const size_t plane = (((size_t)t.b * p.K + p.k) * p.N + (nok[g] ? n : 0)) * HW;
-    Bp[g] = static_cast<const Tin*>(p.B) + plane;
-    Cp[g] = static_cast<const Tin*>(p.C) + plane;
-    hs[g] = p.hsave + (((size_t)t.b * p.channels + (t.act ? t.d : 0)) * p.N + (nok[g] ? n : 0)) * HW;
   }
   const float Dd = (p.first && t.act && p.Dskip) ? p.Dskip[t.d] : 0.f;
   // this lane's two columns after the reduce-scatters
@@ -391,18 +471,40 @@ __global__ void __launch_bounds__(kWarps * 32) k_main(const Args p) {
     for (int c = 0; c < kCols; ++c) V[g][c] = 0.f;
   }
   float dDacc = 0.f;
+  const int n16c = 2 * p.N;                // 8 channels x N carries, in 16-byte chunks
+  const int n16h = 16 * p.N;               // 8 channels x N states x 8 columns
 
-  for (int ii = p.H - 1; ii >= 0; --ii) {
+  // stage one row (scan-order ii) into buf: inputs from pf, carries and h of row ii-1 by cp.async
+  auto stage_ws = [&](float* buf, int ii) {
     const int i = row_of(p, ii);
-    float xv[kCols], dl[kCols], gy[kCols];
-    if (t.act) {
-      load8(xm + (size_t)i * p.W, t.j0, p.W, p.vec_in, xv);
-      load8(dm + (size_t)i * p.W, t.j0, p.W, p.vec_in, dl);
-      load8(gm + (size_t)i * p.W, t.j0, p.W, p.vec_g, gy);
-    } else {
-#pragma unroll
-      for (int c = 0; c < kCols; ++c) xv[c] = dl[c] = gy[c] = 0.f;
+    const size_t c0 = carry_idx(p, t.b, t.cgi * kCh, i, t.s, 0);
+    copy_block(buf + kOffCF, p.cf + c0, n16c, lane);
+    copy_block(buf + kOffCB, p.cb + c0, n16c, lane);
+    if (ii > 0) copy_block(buf + kOffH, p.hsave + hs_idx(p, t.b, t.cgi * kCh, row_of(p, ii - 1), t.s, 0), n16h, lane);
+  };
+  InputPrefetch<Tin, Tg, NG, true, true> pf;
+  pf.init(p, t, lane);
+  pf.load(p, row_of(p, p.H - 1));
+  stage_ws(buf0, p.H - 1);
+  cp_commit();
+  pf.store(buf0, lane);
+
+  for (int e = 0; e < p.H; ++e) {
+    const int ii = p.H - 1 - e;
+    const int i = row_of(p, ii);
+    float* cur = buf0 + (e & 1) * kBufMain;
+    float* nxt = buf0 + ((e + 1) & 1) * kBufMain;
+    if (ii > 0) {
+      pf.load(p, row_of(p, ii - 1));
+      stage_ws(nxt, ii - 1);
     }
+    cp_commit();
+    cp_wait1();
+    __syncwarp();
+    float xv[kCols], dl[kCols], gy[kCols];
+    lds8(cur + kOffX + cg * kCols, xv);
+    lds8(cur + kOffD + cg * kCols, dl);
+    lds8(cur + kOffG + cg * kCols, gy);
     float dxp[kCols];
 #pragma unroll
     for (int c = 0; c < kCols; ++c) {
@@ -415,32 +517,24 @@ __global__ void __launch_bounds__(kWarps * 32) k_main(const Args p) {
 
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
+      const int n = t.q + 4 * g;
       const bool live = t.act && nok[g];
       float bv[kCols], cv[kCols], hp[kCols];
-      float hin = 0.f, cin = 0.f;
-      if (nok[g]) {
-        load8(Bp[g] + (size_t)i * p.W, t.j0, p.W, p.vec_in, bv);
-        load8(Cp[g] + (size_t)i * p.W, t.j0, p.W, p.vec_in, cv);
-      } else {
-#pragma unroll
-        for (int c = 0; c < kCols; ++c) bv[c] = cv[c] = 0.f;
-      }
+      lds8(cur + kOffB + n * kCols, bv);
+      lds8(cur + kOffC + n * kCols, cv);
       if (live && ii > 0) {
-        load8_ws(hs[g] + (size_t)row_of(p, ii - 1) * p.W, t.j0, p.W, p.vec_h, hp);
+        lds8(cur + kOffH + (cg * p.N + n) * kCols, hp);
       } else {
 #pragma unroll
         for (int c = 0; c < kCols; ++c) hp[c] = 0.f;
       }
-      if (live) {
-        const size_t ci = carry_idx(p, t.b, t.d, i, t.s, t.q + 4 * g);
-        hin = p.cf[ci];
-        cin = p.cb[ci];
-      }
+      const float hin = live ? cur[kOffCF + cg * p.N + n] : 0.f;
+      const float cin = live ? cur[kOffCB + cg * p.N + n] : 0.f;
       float a[kCols], hhp[kCols], hc[kCols];
       float r = hin;
 #pragma unroll
-      for (int e = 0; e < kCols; ++e) {       // forward: hh before each column, and h
-        const int c = FW ? kCols - 1 - e : e;
+      for (int k = 0; k < kCols; ++k) {       // forward: hh before each column, and h
+        const int c = FW ? kCols - 1 - k : k;
         a[c] = ex2_approx(dl[c] * A2[g]);
         hhp[c] = r;
         r = fmaf(a[c], r, dxp[c] * bv[c]);
@@ -455,8 +549,8 @@ __global__ void __launch_bounds__(kWarps * 32) k_main(const Args p) {
       float pB[kCols], pC[kCols];
       float carry = cin;
 #pragma unroll
-      for (int e = 0; e < kCols; ++e) {       // adjoint, horizontal, and what each column adds
-        const int c = FW ? e : kCols - 1 - e;
+      for (int k = 0; k < kCols; ++k) {       // adjoint, horizontal, and what each column adds
+        const int c = FW ? k : kCols - 1 - k;
         const float ghh = gh[c] + carry;
         carry = a[c] * ghh;
         const float ta = fmaf(gh[c], hp[c], ghh * hhp[c]) * a[c];
@@ -487,8 +581,7 @@ __global__ void __launch_bounds__(kWarps * 32) k_main(const Args p) {
       }
       if (nok[g]) {
         const int j = t.j0 + cbc;
-        float* dst = (hi ? p.dC : p.dB) + (((size_t)t.b * p.K + p.k) * p.N + t.q + 4 * g) * HW +
-                     (size_t)i * p.W + j;
+        float* dst = (hi ? p.dC : p.dB) + (((size_t)t.b * p.K + p.k) * p.N + n) * HW + (size_t)i * p.W + j;
         if (p.vec2 && j + 1 < p.W) {
           atomicAdd(reinterpret_cast<float2*>(dst), make_float2(o[0], o[1]));
         } else {
@@ -519,9 +612,9 @@ __global__ void __launch_bounds__(kWarps * 32) k_main(const Args p) {
       const bool ok0 = j < p.W, ok1 = j + 1 < p.W;
       float vx[2], vd[2];
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        vx[e] = fmaf(pick(dl, m2, m1, e), f1[e], Dd * pick(gy, m2, m1, e));
-        vd[e] = fmaf(pick(xv, m2, m1, e), f1[e], f2[e]);
+      for (int k = 0; k < 2; ++k) {
+        vx[k] = fmaf(pick(dl, m2, m1, k), f1[k], Dd * pick(gy, m2, m1, k));
+        vd[k] = fmaf(pick(xv, m2, m1, k), f1[k], f2[k]);
       }
       const size_t idx = map + (size_t)i * p.W + j;
       if (!p.first) {                         // add what the earlier orientations left
@@ -536,6 +629,8 @@ __global__ void __launch_bounds__(kWarps * 32) k_main(const Args p) {
         put2(p.accd, idx, vd[0], vd[1], ok0, ok1, p.vec2);
       }
     }
+    if (ii > 0) pf.store(nxt, lane);
+    __syncwarp();
   }
 #pragma unroll
   for (int g = 0; g < NG; ++g)
@@ -568,7 +663,8 @@ int bwd_shape(int batch, int channels, int H, int W, int N, unsigned flags, BwdS
   const unsigned long long xy = static_cast<unsigned long long>(batch) * channels * hw;
   const unsigned long long bc = static_cast<unsigned long long>(batch) * K * N * hw;
   const unsigned long long hs = static_cast<unsigned long long>(batch) * channels * N * hw;
-  const unsigned long long cr = static_cast<unsigned long long>(batch) * channels * H * S * N;
+  const int ncg = (channels + kCh - 1) / kCh;
+  const unsigned long long cr = static_cast<unsigned long long>(batch) * ncg * kCh * H * S * N;
   if (xy > (1ull << 40) || bc > (1ull << 40) || hs > (1ull << 40) || cr > (1ull << 40)) return SCAN2D_E_DIMS;
   s->batch = batch; s->channels = channels; s->H = H; s->W = W; s->N = N; s->K = K; s->S = S;
   s->ncg = (channels + kCh - 1) / kCh;
@@ -586,16 +682,18 @@ int bwd_shape(int batch, int channels, int H, int W, int N, unsigned flags, BwdS
 size_t round256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 struct WsLayout {
-  size_t hsave, cf, cb, beta, accx, accd, total;
+  size_t hsave, tf, tb, beta, cf, cb, accx, accd, total;
 };
 
 WsLayout ws_layout(const BwdShape& s) {
   WsLayout l{};
   size_t off = 0;
-  l.hsave = off; off += round256(s.xy * s.N * sizeof(float));
+  l.hsave = off; off += round256(s.carries * kCols * sizeof(float));   // strips padded to 8 columns
+  l.tf = off;    off += round256(s.carries * sizeof(float));
+  l.tb = off;    off += round256(s.carries * sizeof(float));
+  l.beta = off;  off += round256(s.carries * sizeof(float));
   l.cf = off;    off += round256(s.carries * sizeof(float));
   l.cb = off;    off += round256(s.carries * sizeof(float));
-  l.beta = off;  off += round256(s.carries * sizeof(float));
   const bool acc = !s.out_f32 && s.K > 1;    // bf16 outputs summed over orientations in fp32
   l.accx = off;  off += acc ? round256(s.xy * sizeof(float)) : 0;
   l.accd = off;  off += acc ? round256(s.xy * sizeof(float)) : 0;
@@ -605,18 +703,32 @@ WsLayout ws_layout(const BwdShape& s) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+template <typename K>
+bool launch_warps(K kern, int floats_per_buffer, const Args& a, cudaStream_t st) {
+  const unsigned blocks = static_cast<unsigned>((a.tasks + kWarps - 1) / kWarps);
+  const size_t smem = static_cast<size_t>(kWarps) * 2 * floats_per_buffer * sizeof(float);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+    return false;
+  kern<<<blocks, kWarps * 32, smem, st>>>(a);
+  return true;
+}
+
 template <typename Tin, typename Tg, int NG>
 int launch_orientation(const Args& a, bool fw, cudaStream_t st) {
-  const unsigned blocks = static_cast<unsigned>((a.tasks + kWarps - 1) / kWarps);
-  const long long threads = (long long)a.batch * a.channels * a.H * a.N;
+  const long long threads = (long long)a.batch * a.H * a.ncg * kCh * a.N;
   const unsigned cblocks = static_cast<unsigned>((threads + 255) / 256);
-  if (fw) k_pre<Tin, Tg, NG, true><<<blocks, kWarps * 32, 0, st>>>(a);
-  else k_pre<Tin, Tg, NG, false><<<blocks, kWarps * 32, 0, st>>>(a);
+  bool ok = fw ? launch_warps(k_pre<Tin, Tg, NG, true>, kBufPre, a, st)
+               : launch_warps(k_pre<Tin, Tg, NG, false>, kBufPre, a, st);
   k_carry<<<cblocks, 256, 0, st>>>(a, fw ? 1 : 0);
-  if (fw) k_states<Tin, NG, true><<<blocks, kWarps * 32, 0, st>>>(a);
-  else k_states<Tin, NG, false><<<blocks, kWarps * 32, 0, st>>>(a);
-  if (fw) k_main<Tin, Tg, NG, true><<<blocks, kWarps * 32, 0, st>>>(a);
-  else k_main<Tin, Tg, NG, false><<<blocks, kWarps * 32, 0, st>>>(a);
+  ok = ok && (fw ? launch_warps(k_states<Tin, NG, true>, kBufStates, a, st)
+                 : launch_warps(k_states<Tin, NG, false>, kBufStates, a, st));
+  ok = ok && (fw ? launch_warps(k_main<Tin, Tg, NG, true>, kBufMain, a, st)
+                 : launch_warps(k_main<Tin, Tg, NG, false>, kBufMain, a, st));
+  if (!ok) {
+    cudaGetLastError();
+    return SCAN2D_E_LAUNCH;
+  }
   return cudaGetLastError() == cudaSuccess ? SCAN2D_OK : SCAN2D_E_LAUNCH;
 }
 
@@ -678,16 +790,17 @@ int scan2d_bwd(const void* x, const void* delta, const float* A, const void* B, 
   a.accd = s.out_f32 ? static_cast<float*>(ddelta) : reinterpret_cast<float*>(ws + l.accd);
   a.dA = dA; a.dB = dB; a.dC = dC; a.dDskip = dDskip;
   a.hsave = reinterpret_cast<float*>(ws + l.hsave);
+  a.tf = reinterpret_cast<float*>(ws + l.tf);
+  a.tb = reinterpret_cast<float*>(ws + l.tb);
+  a.beta = reinterpret_cast<float*>(ws + l.beta);
   a.cf = reinterpret_cast<float*>(ws + l.cf);
   a.cb = reinterpret_cast<float*>(ws + l.cb);
-  a.beta = reinterpret_cast<float*>(ws + l.beta);
   a.batch = batch; a.channels = channels; a.H = H; a.W = W; a.N = N; a.K = s.K; a.S = s.S;
   a.ncg = s.ncg;
   a.tasks = (long long)batch * s.S * s.ncg;
   const size_t row_in = (size_t)W * s.in_elem, row_out = (size_t)W * s.out_elem;
   a.vec_in = row_in % 16 == 0 && aligned(x, 16) && aligned(delta, 16) && aligned(B, 16) && aligned(C, 16);
   a.vec_g = row_out % 16 == 0 && aligned(dy, 16);
-  a.vec_h = W % 4 == 0;
   a.vec2 = W % 2 == 0 && aligned(dx, 2 * s.out_elem) && aligned(ddelta, 2 * s.out_elem) &&
            aligned(dB, 8) && aligned(dC, 8);
 

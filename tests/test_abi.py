@@ -121,10 +121,11 @@ def test_bwd_workspace_size_and_host_checks(lib):
     m = _header_macros()
     assert lib.SCAN2D_E_WORKSPACE == m["SCAN2D_E_WORKSPACE"]
     assert lib.SCAN2D_BWD_MAX_N == m["SCAN2D_BWD_MAX_N"]
-    # hsave: N floats per element (4 * 64 * 4); three strip-carry arrays of H * strips * N
-    # floats per channel (8 * 1 * 4 * 4 channels), each rounded up to 256 bytes
+    # channels are padded to a group of 8; hsave: N floats per element of strips padded to 8
+    # columns (8 channels * 64 * 4 states * 4 bytes); five strip-carry arrays of H * strips * N
+    # floats per channel (8 * 1 * 4 * 8 channels * 4 bytes), each rounded up to 256 bytes
     n = lib.scan2d_bwd_workspace_bytes(1, 4, 8, 8, 4, 0x10)
-    assert n == 4 * 64 * 4 * 4 + 3 * 512
+    assert n == 8 * 64 * 4 * 4 + 5 * 8 * 4 * 8 * 4
     # bf16 y with several orientations adds two fp32 accumulators of the element count
     nb = lib.scan2d_bwd_workspace_bytes(1, 4, 8, 8, 4, 0x31)
     assert nb == n + 2 * 4 * 64 * 4
