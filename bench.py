@@ -2,7 +2,9 @@
 the fraction of the kernel's roofline.  One JSON line on rank 0.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload giga|vision|small|wsi|tiny]
-                    [--impl ours|reference] [--no-cpu-baseline] [--others]
+                    [--impl ours|reference] [--no-cpu-baseline] [--others] [--pass fwd|bwd]
+
+--pass bwd times the gradients (scan2d_bwd, one call per step) on the same workloads instead.
 
 A step is one scan2d_fwd call over one batch of the workload (every step of the path runs
 in it).  N > 1 runs under torchrun, one rank per GPU; the (b, d) maps are independent, so
@@ -67,6 +69,28 @@ def roofline_model(w: inputs.Workload):
 
 
 METRIC = "2D selective-scan fwd Gelem/s (B*D*H*W) and % of HBM/SFU roofline"
+METRIC_BWD = "2D selective-scan bwd Gelem/s (B*D*H*W) and % of roofline"
+
+
+def roofline_model_bwd(w: inputs.Workload):
+    """Algorithmic work per element of the gradients: every input and the cotangent read
+    once, every gradient written once, Abar once per (position, state), and per (element,
+    state, orientation) the adjoint's fp32 work: Abar's argument, the forward horizontal
+    and vertical updates with Bbar x, the two adjoint updates (FMA and multiply each), and
+    the five products and three sums that feed dx, ddelta, dA, dB, dC (16 operations)."""
+    s = 2 if w.dtype == "bf16" else 4
+    bytes_el = 3 * s + 2 * s + w.K * 2 * w.N * (s + 4) / w.channels
+    exps_el = w.N
+    fp32_el = 16 * w.N * w.K + 4
+    hbm_gbs, hbm_kind, sm_mhz = _peaks()
+    clk = sm_mhz * 1e6
+    t_hbm = bytes_el / (hbm_gbs * 1e9)
+    t_sfu = exps_el / (SMS * MUFU_PER_CLK_SM * clk)
+    t_fp32 = fp32_el / (SMS * FP32_PER_CLK_SM * clk)
+    bound = max((t_hbm, "hbm"), (t_sfu, "sfu"), (t_fp32, "fp32"))[1]
+    return dict(bytes_el=bytes_el, exps_el=exps_el, fp32_el=fp32_el, t_hbm=t_hbm, t_sfu=t_sfu,
+                t_fp32=t_fp32, bound=bound, hbm_gbs=hbm_gbs, hbm_kind=hbm_kind, sm_mhz=sm_mhz,
+                roof_gelem=1e-9 / max(t_hbm, t_sfu, t_fp32))
 
 
 def base_config(w: inputs.Workload, world: int) -> dict:
@@ -320,6 +344,110 @@ def measure_e2e(w, d, torch, scan2d, device, flags, steps):
     return dict(ms=ms, steps=n, h2d=h2d, d2h=d2h)
 
 
+def measure_backward(w, torch, scan2d, device, seed, steps, warmup):
+    """scan2d_bwd on device-resident inputs and cotangent, one caller-owned workspace."""
+    d = inputs.make_inputs(w, seed=seed)
+    dy = inputs.make_cotangent(w, seed=seed)
+    flags = scan2d.flags_for(w.dtype == "bf16", w.orient_mask)
+    t = {k: _to_dev(d[k], torch, device) for k in ("x", "delta", "A", "B", "C", "Dskip")}
+    t["dy"] = _to_dev(dy, torch, device)
+    set_bytes = sum(v.numel() * v.element_size() for v in t.values() if v is not None)
+    n_sets = max(1, math.ceil(3 * L2_BYTES / set_bytes))
+    sets = [t] + [{k: (v.clone() if v is not None else None) for k, v in t.items()} for _ in range(n_sets - 1)]
+    ws = torch.empty(scan2d.scan2d_bwd_workspace_bytes(w.batch, w.channels, w.H, w.W, w.N, flags),
+                     dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        s = sets[i % n_sets]
+        return scan2d.scan2d_bwd(s["x"], s["delta"], s["A"], s["B"], s["C"], s["Dskip"], s["dy"],
+                                 flags=flags, workspace=ws, stream=stream)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index) as clk:
+        e0.record(stream)
+        for i in range(steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    err = scan2d.scan2d_get_device_error()
+    if err:
+        raise RuntimeError(f"device error {err}: {scan2d.scan2d_strerror(err)}")
+    return dict(ms=ms, n_sets=n_sets, clocks=clk.summary(), d=d, dy=dy, ws_bytes=ws.numel())
+
+
+def _oracle_bwd_sample_rate(w: inputs.Workload, d: dict, dy, budget_s: float):
+    """Time the fp64 oracle's gradients on whole maps (one batch element, growing channel
+    counts) until the budget is used."""
+    import oracle
+    oracle.build()
+    dyf = inputs.bf16_bits_to_f32(dy).astype(np.float64) if dy.dtype == np.uint16 else dy.astype(np.float64)
+    elems, t_used, ch = 0, 0.0, 1
+    while True:
+        sub = slice(0, min(ch, w.channels))
+        t0 = time.perf_counter()
+        oracle.scan2d_bwd(d["x"][:1, sub], d["delta"][:1, sub], d["A"][sub], d["B"][:1], d["C"][:1],
+                          None if d["Dskip"] is None else d["Dskip"][sub], dyf[:1, sub], d["orient_mask"])
+        t_used += time.perf_counter() - t0
+        elems += (sub.stop - sub.start) * w.H * w.W
+        if t_used >= budget_s or ch >= w.channels:
+            break
+        ch *= 2
+    return elems / t_used / 1e9, elems, t_used
+
+
+def run_backward(args, w):
+    import torch
+    from selective_state_space_scan2d_b200 import scan2d
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+        torch.distributed.barrier()
+    res = measure_backward(w, torch, scan2d, device, seed=rank, steps=args.steps, warmup=args.warmup)
+    (ms,) = max_over_ranks([res["ms"]], device=device)
+    value = whole_job_gelem(w.elements, world, ms)
+    rm = roofline_model_bwd(w)
+    if rm["bound"] == "sfu":
+        achieved, peak, unit = w.elements * rm["exps_el"] / (ms * 1e-3) / 1e9, SMS * MUFU_PER_CLK_SM * rm["sm_mhz"] * 1e-3, "Gex2/s"
+    elif rm["bound"] == "fp32":
+        achieved, peak, unit = w.elements * rm["fp32_el"] / (ms * 1e-3) / 1e9, SMS * FP32_PER_CLK_SM * rm["sm_mhz"] * 1e-3, "Gfp32op/s"
+    else:
+        achieved, peak, unit = w.elements * rm["bytes_el"] / (ms * 1e-3) / 1e9, rm["hbm_gbs"], "GB/s"
+    launches = 4 * w.K
+    line = {
+        "metric": METRIC_BWD, "value": value, "unit": "Gelem/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32" if w.dtype == "f32" else "bf16-in/f32-acc", "data": "synthetic",
+        "config": {**base_config(w, world), "pass": "bwd",
+                   "l2": f"inputs rotated over {res['n_sets']} device copies (> 3x L2 per rotation)",
+                   "workspace_bytes": res["ws_bytes"]},
+        "roofline": {"bound": "alu" if rm["bound"] != "hbm" else "hbm", "unit_of_bound": rm["bound"],
+                     "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                     "traffic": None, "scope": f"whole scan2d_bwd call ({launches} kernel launches)",
+                     "roofline_gelem_s": rm["roof_gelem"]},
+        "clocks": res["clocks"], "gpu_launches": args.steps * launches,
+        "e2e": None,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, elems, secs = _oracle_bwd_sample_rate(w, res["d"], res["dy"], args.cpu_budget)
+        line["cpu_baseline"] = {"value": rate, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
+                                "sample": f"gradients of whole maps of batch element 0 of {w.name} ({elems} elements) in {secs:.1f} s, fp64 C oracle, 1 thread"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -333,6 +461,8 @@ def main():
     ap.add_argument("--override", action="append", default=[], metavar="KEY=INT",
                     help="change batch/channels/H/W of the workload (smaller cases for ncu captures)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer (e2e) leg")
+    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"],
+                    help="bwd: time the gradients (scan2d_bwd) instead of the forward")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -348,6 +478,9 @@ def main():
 
     if args.impl == "reference":
         run_reference(args, w)
+        return
+    if args.which == "bwd":
+        run_backward(args, w)
         return
 
     import torch

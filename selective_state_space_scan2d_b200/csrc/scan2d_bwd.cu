@@ -89,10 +89,11 @@ __device__ __forceinline__ float ex2_approx(float v) {
 __device__ __forceinline__ float to_f(float v) { return v; }
 __device__ __forceinline__ float to_f(uint16_t v) { return __uint_as_float(static_cast<uint32_t>(v) << 16); }
 
-// One of the lane's 8 columns, chosen by two lane bits (keeps the register arrays static).
-__device__ __forceinline__ float pick(const float (&v)[kCols], bool m2, bool m1, int e) {
-  const float lo = m1 ? v[2 + e] : v[e];
-  const float hi = m1 ? v[6 + e] : v[4 + e];
+// One of the lane's 8 columns (held as 4 pairs), chosen by two lane bits (keeps the register
+// arrays static): column (m2 ? 4 : 0) + (m1 ? 2 : 0) + e.
+__device__ __forceinline__ float pick(const float2 (&v)[4], bool m2, bool m1, int e) {
+  const float lo = m1 ? (e ? v[1].y : v[1].x) : (e ? v[0].y : v[0].x);
+  const float hi = m1 ? (e ? v[3].y : v[3].x) : (e ? v[2].y : v[2].x);
   return m2 ? hi : lo;
 }
 
@@ -141,6 +142,18 @@ __device__ __forceinline__ void lds8(const float* src, float (&v)[kCols]) {
   v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
   v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
+
+constexpr int kPairs = kCols / 2;
+
+// 8 floats from shared memory as 4 column pairs
+__device__ __forceinline__ void lds8x2(const float* src, float2 (&v)[kPairs]) {
+  const float4 a = *reinterpret_cast<const float4*>(src);
+  const float4 b = *reinterpret_cast<const float4*>(src + 4);
+  v[0] = make_float2(a.x, a.y); v[1] = make_float2(a.z, a.w);
+  v[2] = make_float2(b.x, b.y); v[3] = make_float2(b.z, b.w);
+}
+
+__device__ __forceinline__ float lo_hi(const float2 (&v)[kPairs], int c) { return (c & 1) ? v[c >> 1].y : v[c >> 1].x; }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -283,6 +296,7 @@ __global__ void __launch_bounds__(kWarps * 32) k_pre(const Args p) {
       for (int c = 0; c < kCols; ++c) {
         a[c] = ex2_approx(dl[c] * A2[g]);
         prod *= a[c];
+        V[g][c] = a[c] * fmaf(cv[c], gy[c], V[g][c]);   // a*gh of this row
       }
       float r = 0.f;                        // forward: hh leaving the strip, from zero
 #pragma unroll
@@ -294,9 +308,7 @@ __global__ void __launch_bounds__(kWarps * 32) k_pre(const Args p) {
 #pragma unroll
       for (int k = 0; k < kCols; ++k) {
         const int c = FW ? k : kCols - 1 - k;
-        const float gh = fmaf(cv[c], gy[c], V[g][c]);
-        V[g][c] = a[c] * gh;
-        hc = a[c] * (gh + hc);
+        hc = fmaf(a[c], hc, V[g][c]);       // a*(gh + hc)
       }
       if (t.act && nok[g]) {
         const size_t ci = carry_idx(p, t.b, t.d, i, t.s, t.q + 4 * g);
@@ -355,7 +367,7 @@ __global__ void __launch_bounds__(256) k_carry(const Args p, int fw) {
 
 // ---- 3. forward vertical state of every element -----------------------------------------------
 template <typename Tin, int NG, bool FW>
-__global__ void __launch_bounds__(kWarps * 32) k_states(const Args p) {
+__global__ void __launch_bounds__(kWarps * 32, 2) k_states(const Args p) {
   extern __shared__ __align__(16) float smem[];
   Task t;
   if (!decode(p, t)) return;
@@ -369,11 +381,11 @@ __global__ void __launch_bounds__(kWarps * 32) k_states(const Args p) {
     nok[g] = n < p.N;
     A2[g] = (t.act && nok[g]) ? p.A[(size_t)t.d * p.N + n] * kLog2e : 0.f;
   }
-  float h[NG][kCols];
+  float2 h[NG][kPairs];
 #pragma unroll
   for (int g = 0; g < NG; ++g)
 #pragma unroll
-    for (int c = 0; c < kCols; ++c) h[g][c] = 0.f;
+    for (int k = 0; k < kPairs; ++k) h[g][k] = make_float2(0.f, 0.f);
   const int n16 = 2 * p.N;                 // 8 channels x N carries, in 16-byte chunks
 
   InputPrefetch<Tin, float, NG, false, false> pf;
@@ -393,23 +405,37 @@ __global__ void __launch_bounds__(kWarps * 32) k_states(const Args p) {
     cp_commit();
     cp_wait1();
     __syncwarp();
-    float xv[kCols], dl[kCols];
-    lds8(cur + kOffX + cg * kCols, xv);
-    lds8(cur + kOffD + cg * kCols, dl);
+    float2 xv[kPairs], dl[kPairs], dxp[kPairs];
+    lds8x2(cur + kOffX + cg * kCols, xv);
+    lds8x2(cur + kOffD + cg * kCols, dl);
+#pragma unroll
+    for (int k = 0; k < kPairs; ++k) dxp[k] = __fmul2_rn(dl[k], xv[k]);
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
       const int n = t.q + 4 * g;
-      float bv[kCols];
-      lds8(cur + kOffB + n * kCols, bv);
+      float2 bv[kPairs], a[kPairs], u[kPairs], rr[kPairs];
+      lds8x2(cur + kOffB + n * kCols, bv);
+      const float2 A2g = make_float2(A2[g], A2[g]);
+#pragma unroll
+      for (int k = 0; k < kPairs; ++k) {
+        const float2 arg = __fmul2_rn(dl[k], A2g);
+        a[k] = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+        u[k] = __fmul2_rn(dxp[k], bv[k]);
+      }
       float r = nok[g] ? cur[kOffCF + cg * p.N + n] : 0.f;
 #pragma unroll
-      for (int k = 0; k < kCols; ++k) {
+      for (int k = 0; k < kCols; ++k) {       // horizontal, in scan order
         const int c = FW ? kCols - 1 - k : k;
-        const float a = ex2_approx(dl[c] * A2[g]);
-        r = fmaf(a, r, (dl[c] * xv[c]) * bv[c]);
-        h[g][c] = fmaf(a, h[g][c], r);
+        r = fmaf(lo_hi(a, c), r, lo_hi(u, c));
+        if (c & 1) rr[c >> 1].y = r; else rr[c >> 1].x = r;
       }
-      if (t.act && nok[g]) st8(p.hsave + hs_idx(p, t.b, t.d, i, t.s, n), h[g]);
+#pragma unroll
+      for (int k = 0; k < kPairs; ++k) h[g][k] = __ffma2_rn(a[k], h[g][k], rr[k]);   // vertical
+      if (t.act && nok[g]) {
+        float* dst = p.hsave + hs_idx(p, t.b, t.d, i, t.s, n);
+        *reinterpret_cast<float4*>(dst) = make_float4(h[g][0].x, h[g][0].y, h[g][1].x, h[g][1].y);
+        *reinterpret_cast<float4*>(dst + 4) = make_float4(h[g][2].x, h[g][2].y, h[g][3].x, h[g][3].y);
+      }
     }
     if (ii + 1 < p.H) pf.store(nxt, lane);
     __syncwarp();
@@ -462,13 +488,13 @@ __global__ void __launch_bounds__(kWarps * 32) k_main(const Args p) {
   // this lane's two columns after the reduce-scatters
   const int cq = (m2 ? 4 : 0) + (m1 ? 2 : 0);           // per-element outputs
   const int cbc = (m8 ? 4 : 0) + (m4 ? 2 : 0);          // dB / dC
-  float V[NG][kCols];
-  float dAacc[NG];
+  float2 V[NG][kPairs];
+  float2 dAacc[NG];
 #pragma unroll
   for (int g = 0; g < NG; ++g) {
-    dAacc[g] = 0.f;
+    dAacc[g] = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int c = 0; c < kCols; ++c) V[g][c] = 0.f;
+    for (int k = 0; k < kPairs; ++k) V[g][k] = make_float2(0.f, 0.f);
   }
   float dDacc = 0.f;
   const int n16c = 2 * p.N;                // 8 channels x N carries, in 16-byte chunks
@@ -501,64 +527,76 @@ __global__ void __launch_bounds__(kWarps * 32) k_main(const Args p) {
     cp_commit();
     cp_wait1();
     __syncwarp();
-    float xv[kCols], dl[kCols], gy[kCols];
-    lds8(cur + kOffX + cg * kCols, xv);
-    lds8(cur + kOffD + cg * kCols, dl);
-    lds8(cur + kOffG + cg * kCols, gy);
-    float dxp[kCols];
+    float2 xv[kPairs], dl[kPairs], gy[kPairs], dxp[kPairs];
+    lds8x2(cur + kOffX + cg * kCols, xv);
+    lds8x2(cur + kOffD + cg * kCols, dl);
+    lds8x2(cur + kOffG + cg * kCols, gy);
+    float2 dD2 = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int c = 0; c < kCols; ++c) {
-      dxp[c] = dl[c] * xv[c];
-      dDacc = fmaf(gy[c], xv[c], dDacc);
+    for (int k = 0; k < kPairs; ++k) {
+      dxp[k] = __fmul2_rn(dl[k], xv[k]);
+      dD2 = __ffma2_rn(gy[k], xv[k], dD2);
     }
-    float s1[kCols], s2[kCols];              // sum over the lane's states of ghh*B and dL/da*a*A
+    dDacc += dD2.x + dD2.y;
+    float2 s1[kPairs], s2[kPairs];           // sum over the lane's states of ghh*B and dL/da*a*A
 #pragma unroll
-    for (int c = 0; c < kCols; ++c) s1[c] = s2[c] = 0.f;
+    for (int k = 0; k < kPairs; ++k) s1[k] = s2[k] = make_float2(0.f, 0.f);
 
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
       const int n = t.q + 4 * g;
       const bool live = t.act && nok[g];
-      float bv[kCols], cv[kCols], hp[kCols];
-      lds8(cur + kOffB + n * kCols, bv);
-      lds8(cur + kOffC + n * kCols, cv);
+      float2 bv[kPairs], cv[kPairs], hp[kPairs];
+      lds8x2(cur + kOffB + n * kCols, bv);
+      lds8x2(cur + kOffC + n * kCols, cv);
       if (live && ii > 0) {
-        lds8(cur + kOffH + (cg * p.N + n) * kCols, hp);
+        lds8x2(cur + kOffH + (cg * p.N + n) * kCols, hp);
       } else {
 #pragma unroll
-        for (int c = 0; c < kCols; ++c) hp[c] = 0.f;
+        for (int k = 0; k < kPairs; ++k) hp[k] = make_float2(0.f, 0.f);
       }
       const float hin = live ? cur[kOffCF + cg * p.N + n] : 0.f;
       const float cin = live ? cur[kOffCB + cg * p.N + n] : 0.f;
-      float a[kCols], hhp[kCols], hc[kCols];
+      const float2 A2g = make_float2(A2[g], A2[g]);
+      const float2 Afg = make_float2(Af[g], Af[g]);
+      float2 a[kPairs], u[kPairs], gh[kPairs];
+#pragma unroll
+      for (int k = 0; k < kPairs; ++k) {
+        const float2 arg = __fmul2_rn(dl[k], A2g);
+        a[k] = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+        u[k] = __fmul2_rn(dxp[k], bv[k]);
+        gh[k] = __ffma2_rn(cv[k], gy[k], V[g][k]);          // adjoint, vertical
+        V[g][k] = __fmul2_rn(a[k], gh[k]);
+      }
+      float2 hhp[kPairs], rr[kPairs], cpre[kPairs];
       float r = hin;
 #pragma unroll
-      for (int k = 0; k < kCols; ++k) {       // forward: hh before each column, and h
+      for (int k = 0; k < kCols; ++k) {       // forward recompute: hh before and after each column
         const int c = FW ? kCols - 1 - k : k;
-        a[c] = ex2_approx(dl[c] * A2[g]);
-        hhp[c] = r;
-        r = fmaf(a[c], r, dxp[c] * bv[c]);
-        hc[c] = fmaf(a[c], hp[c], r);
+        if (c & 1) hhp[c >> 1].y = r; else hhp[c >> 1].x = r;
+        r = fmaf(lo_hi(a, c), r, lo_hi(u, c));
+        if (c & 1) rr[c >> 1].y = r; else rr[c >> 1].x = r;
       }
-      float gh[kCols];
-#pragma unroll
-      for (int c = 0; c < kCols; ++c) {       // adjoint, vertical
-        gh[c] = fmaf(cv[c], gy[c], V[g][c]);
-        V[g][c] = a[c] * gh[c];
-      }
-      float pB[kCols], pC[kCols];
       float carry = cin;
 #pragma unroll
-      for (int k = 0; k < kCols; ++k) {       // adjoint, horizontal, and what each column adds
+      for (int k = 0; k < kCols; ++k) {       // adjoint, horizontal: carry before each column
         const int c = FW ? k : kCols - 1 - k;
-        const float ghh = gh[c] + carry;
-        carry = a[c] * ghh;
-        const float ta = fmaf(gh[c], hp[c], ghh * hhp[c]) * a[c];
-        s1[c] = fmaf(ghh, bv[c], s1[c]);
-        s2[c] = fmaf(ta, Af[g], s2[c]);
-        dAacc[g] = fmaf(ta, dl[c], dAacc[g]);
-        pB[c] = ghh * dxp[c];
-        pC[c] = gy[c] * hc[c];
+        if (c & 1) cpre[c >> 1].y = carry; else cpre[c >> 1].x = carry;
+        carry = fmaf(lo_hi(a, c), carry, lo_hi(V[g], c));  // a*(gh + carry)
+      }
+      float pB[kCols], pC[kCols];
+#pragma unroll
+      for (int k = 0; k < kPairs; ++k) {       // what each column adds
+        const float2 hc = __ffma2_rn(a[k], hp[k], rr[k]);   // h of this row
+        const float2 ghh = __fadd2_rn(gh[k], cpre[k]);
+        const float2 ta = __fmul2_rn(__ffma2_rn(gh[k], hp[k], __fmul2_rn(ghh, hhp[k])), a[k]);
+        s1[k] = __ffma2_rn(ghh, bv[k], s1[k]);
+        s2[k] = __ffma2_rn(ta, Afg, s2[k]);
+        dAacc[g] = __ffma2_rn(ta, dl[k], dAacc[g]);
+        const float2 b2 = __fmul2_rn(ghh, dxp[k]);
+        const float2 c2 = __fmul2_rn(gy[k], hc);
+        pB[2 * k] = b2.x; pB[2 * k + 1] = b2.y;
+        pC[2 * k] = c2.x; pC[2 * k + 1] = c2.y;
       }
       // dB, dC: sum over the warp's 8 channels (lanes xor 16, 8, 4 share the state)
       float k1[kCols];
@@ -594,10 +632,10 @@ __global__ void __launch_bounds__(kWarps * 32) k_main(const Args p) {
     float a1[4], a2[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      const float send1 = m2 ? s1[c] : s1[c + 4];
-      const float send2 = m2 ? s2[c] : s2[c + 4];
-      a1[c] = (m2 ? s1[c + 4] : s1[c]) + __shfl_xor_sync(kFull, send1, 2);
-      a2[c] = (m2 ? s2[c + 4] : s2[c]) + __shfl_xor_sync(kFull, send2, 2);
+      const float s1lo = lo_hi(s1, c), s1hi = lo_hi(s1, c + 4);
+      const float s2lo = lo_hi(s2, c), s2hi = lo_hi(s2, c + 4);
+      a1[c] = (m2 ? s1hi : s1lo) + __shfl_xor_sync(kFull, m2 ? s1lo : s1hi, 2);
+      a2[c] = (m2 ? s2hi : s2lo) + __shfl_xor_sync(kFull, m2 ? s2lo : s2hi, 2);
     }
     float f1[2], f2[2];
 #pragma unroll
@@ -634,7 +672,7 @@ __global__ void __launch_bounds__(kWarps * 32) k_main(const Args p) {
   }
 #pragma unroll
   for (int g = 0; g < NG; ++g)
-    if (t.act && nok[g]) atomicAdd(p.dA + (size_t)t.d * p.N + t.q + 4 * g, dAacc[g]);
+    if (t.act && nok[g]) atomicAdd(p.dA + (size_t)t.d * p.N + t.q + 4 * g, dAacc[g].x + dAacc[g].y);
   if (p.first && t.act && t.q == 0 && p.dDskip) atomicAdd(p.dDskip + t.d, dDacc);
 }
 
