@@ -4,7 +4,8 @@ the fraction of the kernel's roofline.  One JSON line on rank 0.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload giga|vision|small|wsi|tiny]
                     [--impl ours|reference] [--no-cpu-baseline] [--others] [--pass fwd|bwd]
 
---pass bwd times the gradients (scan2d_bwd, one call per step) on the same workloads instead.
+--pass bwd times the gradients (scan2d_bwd, one call per step) on the same workloads instead;
+--pass wsi --workload wsi times the whole-slide path built from a bag of patch features.
 
 A step is one scan2d_fwd call over one batch of the workload (every step of the path runs
 in it).  N > 1 runs under torchrun, one rank per GPU; the (b, d) maps are independent, so
@@ -448,6 +449,83 @@ def run_backward(args, w):
         torch.distributed.destroy_process_group()
 
 
+def run_wsi(args, w):
+    """The whole-slide path: cell map and map built from a bag of patches, then the scan, as
+    two steps (grid gather + scan2d_fwd) and fused (scan2d_fwd_wsi reads x through the cell
+    map).  value = the fused path's Gelem/s; the grid gather's HBM roofline is reported."""
+    import torch
+    from selective_state_space_scan2d_b200 import scan2d
+    if w.name != "wsi" and not w.wsi_mask:
+        raise SystemExit("--pass wsi needs a whole-slide workload (--workload wsi)")
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    b = inputs.make_wsi_bag(w, seed=0)
+    t = {k: _to_dev(b[k], torch, device) for k in ("delta", "A", "B", "C", "Dskip", "feat", "pad")}
+    coords = torch.from_numpy(b["coords"]).to(device)
+    flags = scan2d.flags_for(w.dtype == "bf16", w.orient_mask)
+    npatch = b["feat"].shape[0]
+    out_dtype = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    cell = torch.empty(w.H * w.W, dtype=torch.int32, device=device)
+    x = torch.empty((1, w.channels, w.H, w.W), dtype=t["feat"].dtype, device=device)
+    y = torch.empty((1, w.channels, w.H, w.W), dtype=out_dtype, device=device)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=device)   # written between steps
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        total = 0.0
+        with ClockSampler(0) as clk:
+            for _ in range(args.steps):
+                flush.fill_(1)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+                e1.synchronize()
+                total += e0.elapsed_time(e1)
+        return total / args.steps, clk.summary()
+
+    cells_ms, _ = timed(lambda: scan2d.scan2d_grid_cells(coords, w.H, w.W, cell_patch=cell, stream=stream))
+    gather_ms, _ = timed(lambda: scan2d.scan2d_grid_gather(t["feat"], cell, t["pad"], w.H, w.W, x=x, stream=stream))
+
+    def unfused():
+        scan2d.scan2d_grid_gather(t["feat"], cell, t["pad"], w.H, w.W, x=x, stream=stream)
+        scan2d.scan2d_fwd(x, t["delta"], t["A"], t["B"], t["C"], t["Dskip"], y=y, flags=flags, stream=stream)
+
+    def fused():
+        scan2d.scan2d_fwd_wsi(t["feat"], cell, t["pad"], t["delta"], t["A"], t["B"], t["C"], t["Dskip"],
+                              y=y, flags=flags, stream=stream)
+
+    unfused_ms, _ = timed(unfused)
+    fused_ms, clocks = timed(fused)
+    err = scan2d.scan2d_get_device_error()
+    if err:
+        raise RuntimeError(f"device error {err}")
+    s = 2 if w.dtype == "bf16" else 4
+    gather_bytes = npatch * w.channels * s + w.H * w.W * 4 + w.channels * w.H * w.W * s
+    hbm_gbs, hbm_kind, _ = _peaks()
+    achieved = gather_bytes / (gather_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC + " (whole-slide map read from its bag of patches)",
+        "value": w.elements / (fused_ms * 1e-3) / 1e9, "unit": "Gelem/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": fused_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32" if w.dtype == "f32" else "bf16-in/f32-acc",
+        "data": "synthetic",
+        "config": {**base_config(w, 1), "pass": "wsi", "npatch": npatch,
+                   "l2": "a 252 MB buffer is written before every timed step"},
+        "unfused": {"ms_per_step": unfused_ms, "value": w.elements / (unfused_ms * 1e-3) / 1e9,
+                    "steps": "scan2d_grid_gather + scan2d_fwd"},
+        "grid_cells_ms": cells_ms, "grid_gather_ms": gather_ms,
+        "roofline": {"bound": "hbm", "kernel": "grid gather", "achieved": achieved, "peak": hbm_gbs,
+                     "unit": "GB/s", "frac": achieved / hbm_gbs, "traffic": None,
+                     "algorithmic_bytes": gather_bytes, "peak_kind": f"{hbm_kind} copy bandwidth"},
+        "clocks": clocks, "gpu_launches": args.steps, "e2e": None,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -461,8 +539,8 @@ def main():
     ap.add_argument("--override", action="append", default=[], metavar="KEY=INT",
                     help="change batch/channels/H/W of the workload (smaller cases for ncu captures)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer (e2e) leg")
-    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"],
-                    help="bwd: time the gradients (scan2d_bwd) instead of the forward")
+    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd", "wsi"],
+                    help="bwd: time the gradients (scan2d_bwd); wsi: the whole-slide path from a bag of patches")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -481,6 +559,9 @@ def main():
         return
     if args.which == "bwd":
         run_backward(args, w)
+        return
+    if args.which == "wsi":
+        run_wsi(args, w)
         return
 
     import torch

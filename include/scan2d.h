@@ -140,6 +140,42 @@ int scan2d_fwd_noalloc(const void *x, const void *delta, const float *A, const v
                        int H, int W, int N, unsigned flags, void *stream);
 
 /*
+ * Whole-slide images: the map x built from a bag of patch features ("2DMamba 精读", section
+ * 四.2, the 2DMambaMIL framework, steps 3-4; papernotes.org notes, "方法详解 / 整体框架" and
+ * "关键设计": patch features go back to the 2D grid at the patch's position, and every cell
+ * without a patch holds a learnable non-tissue token p instead of zeros):
+ *     x[d, i, j] = feat[k, d]  if patch k sits at cell (i, j),  else  p[d].
+ *
+ * scan2d_grid_cells -- the cell map of a bag.  coords: device (npatch, 2) int32 (row, column);
+ * cell_patch: device (H*W) int32, written: the index of the patch at each cell, -1 where there
+ * is none.  When several patches name one cell the highest index wins.  Patches outside the
+ * grid are skipped and counted into *n_skipped (device int, written; may be NULL).
+ * Asynchronous on `stream`.  Returns 0, SCAN2D_E_DIMS / _NULL / _ALIGN / _LAUNCH.
+ */
+int scan2d_grid_cells(const int *coords, int npatch, int H, int W, int *cell_patch,
+                      int *n_skipped, void *stream);
+
+/*
+ * scan2d_grid_gather -- writes x (1, channels, H, W) from the bag feat (npatch, channels,
+ * row-major), a cell map and the token pad (channels).  flags: 0 (fp32) or SCAN2D_BF16 (feat,
+ * pad and x bf16).  Cell entries outside [0, npatch) read pad.  Asynchronous on `stream`.
+ * Returns 0, SCAN2D_E_FLAGS / _DIMS / _NULL / _ALIGN / _LAUNCH.
+ */
+int scan2d_grid_gather(const void *feat, const int *cell_patch, const void *pad, void *x,
+                       int npatch, int channels, int H, int W, unsigned flags, void *stream);
+
+/*
+ * scan2d_fwd_wsi -- scan2d_fwd of one map (batch 1) whose x is read from the bag through the
+ * cell map as above, without x being written: the grid step fused in front of the scan.
+ * feat (npatch, channels) and pad (channels) have the element type of x; delta, A, B, C,
+ * Dskip, y, flags as for scan2d_fwd with batch = 1.  Rows are staged by plain loads (no TMA).
+ * Returns the scan2d_fwd codes.
+ */
+int scan2d_fwd_wsi(const void *feat, const int *cell_patch, const void *pad, const void *delta,
+                   const float *A, const void *B, const void *C, const float *Dskip, void *y,
+                   int npatch, int channels, int H, int W, int N, unsigned flags, void *stream);
+
+/*
  * scan2d_query_plan -- how scan2d_fwd would run a call of this shape on a B200 (148
  * multiprocessors, clusters assumed resident), without launching anything or touching a device.  Writes up to n_out (<= SCAN2D_PLAN_FIELDS) values to `out`:
  *   [0] kernel launches per call        [5] columns per warp strip

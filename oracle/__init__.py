@@ -167,5 +167,29 @@ def scan2d_bwd(x, delta, A, B, C, Dskip, dy, orient_mask: int = 1, majorant: boo
     return out
 
 
+def wsi_grid(feat, coords, pad, H: int, W: int):
+    """The map of a whole-slide image from its bag of patches ("2DMamba 精读", section 四.2,
+    the 2DMambaMIL framework, steps 3-4: each patch feature goes back to its grid position;
+    cells without a patch hold the learnable non-tissue token).  Patches are placed in index
+    order, so when two name one cell the later one stays; patches outside the grid are left
+    out and counted.  Returns x (1, channels, H, W) of feat's dtype, the cell map (H*W int32,
+    -1 at non-tissue cells) and the number of patches left out."""
+    feat = np.asarray(feat)
+    npatch, channels = feat.shape
+    cell = np.full((H, W), -1, dtype=np.int32)
+    skipped = 0
+    for k in range(npatch):
+        r, c = int(coords[k][0]), int(coords[k][1])
+        if 0 <= r < H and 0 <= c < W:
+            cell[r, c] = k
+        else:
+            skipped += 1
+    x = np.empty((1, channels, H, W), dtype=feat.dtype)
+    for r in range(H):
+        for c in range(W):
+            x[0, :, r, c] = feat[cell[r, c]] if cell[r, c] >= 0 else pad
+    return x, cell.reshape(-1), skipped
+
+
 def version() -> int:
     return _load().scan2d_oracle_version()

@@ -10,7 +10,7 @@ _BINDING_NAMES = {
     "SCAN2D_BF16", "SCAN2D_OUT_F32", "SCAN2D_OR_TL", "SCAN2D_OR_TR", "SCAN2D_OR_BL",
     "SCAN2D_OR_BR", "scan2d_fwd_noalloc", "SCAN2D_E_SCRATCH", "SCAN2D_NOALLOC_SCRATCH_BYTES",
     "SCAN2D_VFIRST", "scan2d_bwd", "scan2d_bwd_workspace_bytes", "SCAN2D_E_WORKSPACE",
-    "SCAN2D_BWD_MAX_N",
+    "SCAN2D_BWD_MAX_N", "scan2d_grid_cells", "scan2d_grid_gather", "scan2d_fwd_wsi",
 }
 
 

@@ -445,9 +445,12 @@ bool cluster_worth_it(KernelFn fn, int threads, size_t smem, int nseg, int chain
 
 // `fixed_scratch`, when given, is the device address of a buffer of
 // SCAN2D_NOALLOC_SCRATCH_BYTES that replaces the per-stream workspace (nothing is allocated).
+// `cell_patch`, when given, makes x a bag of patch features read through that cell map (one
+// map, batch 1), with `pad` at the cells that hold no patch; such calls stage by plain loads.
 int forward(const void* x, const void* delta, const float* A, const void* B, const void* C,
             const float* Dskip, void* y, int batch, int channels, int H, int W, int N,
-            unsigned flags, cudaStream_t st, char* fixed_scratch = nullptr) {
+            unsigned flags, cudaStream_t st, char* fixed_scratch = nullptr,
+            const int* cell_patch = nullptr, const void* pad = nullptr, int npatch = 0) {
   Shape s;
   int rc = check_shape(batch, channels, H, W, N, flags, &s);
   if (rc) return rc;
@@ -462,7 +465,7 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
   // tensor maps when the layout allows TMA, else the plain-load variant
   TmaMaps tm;
   std::memset(&tm, 0, sizeof tm);
-  bool tma = tma_possible(s, x, delta, B, C);
+  bool tma = cell_patch == nullptr && tma_possible(s, x, delta, B, C);
   CallPlan cp = plan_call(s, tma, true, nsm);
   if (tma) {
     const Plan& p0 = cp.pl;
@@ -486,6 +489,7 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
   Params prm;
   std::memset(&prm, 0, sizeof prm);
   prm.x = x; prm.delta = delta; prm.A = A; prm.B = B; prm.C = C; prm.Dskip = Dskip; prm.y = y;
+  prm.cell_patch = cell_patch; prm.pad = pad; prm.npatch = npatch;
   prm.batch = batch; prm.channels = channels; prm.H = H; prm.W = W; prm.N = N; prm.K = s.K;
   prm.n_cgroups = pl.n_cgroups; prm.n_chains = pl.n_chains;
   prm.strips = pl.strips; prm.wpc = pl.wpc; prm.chains_per_block = pl.chains_per_block;
@@ -620,6 +624,21 @@ int scan2d_fwd_noalloc(const void* x, const void* delta, const float* A, const v
   if (scratch == nullptr) return SCAN2D_E_DEVICE;
   return scan2d::forward(x, delta, A, B, C, Dskip, y, batch, channels, H, W, N, flags,
                          static_cast<cudaStream_t>(stream), scratch);
+}
+
+int scan2d_fwd_wsi(const void* feat, const int* cell_patch, const void* pad, const void* delta,
+                   const float* A, const void* B, const void* C, const float* Dskip, void* y,
+                   int npatch, int channels, int H, int W, int N, unsigned flags, void* stream) {
+  scan2d::Shape s;
+  int rc = scan2d::check_shape(1, channels, H, W, N, flags, &s);
+  if (rc) return rc;
+  if (npatch < 0) return SCAN2D_E_DIMS;
+  if (!cell_patch || !pad || (npatch > 0 && !feat)) return SCAN2D_E_NULL;
+  if (!scan2d::aligned(cell_patch, 4) || !scan2d::aligned(pad, s.in_elem) || !scan2d::aligned(feat, s.in_elem))
+    return SCAN2D_E_ALIGN;
+  // a bag without patches is read at no address; any aligned pointer stands in for it
+  return scan2d::forward(npatch > 0 ? feat : pad, delta, A, B, C, Dskip, y, 1, channels, H, W, N, flags,
+                         static_cast<cudaStream_t>(stream), nullptr, cell_patch, pad, npatch);
 }
 
 int scan2d_query_plan(int batch, int channels, int H, int W, int N, unsigned flags,

@@ -76,7 +76,10 @@ enum Link : int {
 };
 
 struct Params {
-  const void* x;
+  const void* x;            // the map x, or with cell_patch the bag of patch features (npatch, channels)
+  const int* cell_patch;    // null, or (H*W): the bag row at each cell, -1 for a non-tissue cell
+  const void* pad;          // with cell_patch: the non-tissue token (channels)
+  int npatch;               // with cell_patch: rows of the bag (other cell entries read pad)
   const void* delta;
   const float* A;
   const void* B;
@@ -587,8 +590,16 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
         if (region < 2) {
           const int d = grp * L::CPW + rr;
           if (d < p.channels) {
-            const Tin* src = static_cast<const Tin*>(region == 0 ? p.x : p.delta);
-            val = load_raw(src + (static_cast<size_t>(b) * p.channels + d) * HW + static_cast<size_t>(i) * W + col);
+            if (region == 0 && p.cell_patch != nullptr) {
+              // x read from the bag through the cell map (one map, b = 0)
+              const int kp = __ldg(p.cell_patch + static_cast<size_t>(i) * W + col);
+              val = load_raw((kp >= 0 && kp < p.npatch
+                                  ? static_cast<const Tin*>(p.x) + static_cast<size_t>(kp) * p.channels
+                                  : static_cast<const Tin*>(p.pad)) + d);
+            } else {
+              const Tin* src = static_cast<const Tin*>(region == 0 ? p.x : p.delta);
+              val = load_raw(src + (static_cast<size_t>(b) * p.channels + d) * HW + static_cast<size_t>(i) * W + col);
+            }
           }
         } else if (rr < N) {
           const Tin* src = static_cast<const Tin*>(region == 2 ? p.B : p.C);

@@ -27,7 +27,8 @@ import numpy as np
 
 ORIENT_TL, ORIENT_TR, ORIENT_BL, ORIENT_BR = 1, 2, 4, 8
 
-_TENSOR_ID = {"x": 1, "delta": 2, "B": 3, "C": 4, "Dskip": 5, "pad": 6, "mask": 7, "A": 8, "dy": 9}
+_TENSOR_ID = {"x": 1, "delta": 2, "B": 3, "C": 4, "Dskip": 5, "pad": 6, "mask": 7, "A": 8, "dy": 9,
+              "order": 10}
 
 
 @dataclasses.dataclass(frozen=True)
@@ -163,3 +164,25 @@ def make_cotangent(w: Workload | str, seed: int = 0, out_f32: bool = False) -> n
         w = WORKLOADS[w]
     dy = _rng(seed, "dy").standard_normal((w.batch, w.channels, w.H, w.W), dtype=np.float32)
     return f32_to_bf16_bits(dy) if (w.dtype == "bf16" and not out_f32) else dy
+
+
+def make_wsi_bag(w: Workload | str, seed: int = 0) -> dict:
+    """The workload's map as a bag of patches: the tissue cells of make_inputs' mask in a
+    seeded random order, their features feat (npatch, channels) = x at those cells, their
+    coordinates (npatch, 2) int32 (row, column) and the non-tissue token pad (channels), so
+    that placing the bag on the grid gives back make_inputs' x exactly."""
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    if w.batch != 1 or not w.wsi_mask:
+        raise ValueError("a bag describes one whole-slide map (batch 1, wsi_mask)")
+    d = make_inputs(w, seed)
+    mask = wsi_tissue_mask(w.H, w.W, seed)
+    rows, cols = np.nonzero(~mask)
+    order = _rng(seed, "order").permutation(rows.size)
+    rows, cols = rows[order], cols[order]
+    feat = np.ascontiguousarray(d["x"][0][:, rows, cols].T)
+    coords = np.ascontiguousarray(np.stack([rows, cols], axis=1).astype(np.int32))
+    pad = _rng(seed, "pad").standard_normal(w.channels, dtype=np.float32)
+    if w.dtype == "bf16":
+        pad = f32_to_bf16_bits(pad)
+    return dict(d, feat=feat, coords=coords, pad=pad, tissue=~mask)

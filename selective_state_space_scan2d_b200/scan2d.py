@@ -40,6 +40,12 @@ _lib.scan2d_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _v
 _lib.scan2d_bwd.restype = _i
 _lib.scan2d_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _u]
 _lib.scan2d_bwd_workspace_bytes.restype = _sz
+_lib.scan2d_grid_cells.argtypes = [_vp, _i, _i, _i, _vp, _vp, _vp]
+_lib.scan2d_grid_cells.restype = _i
+_lib.scan2d_grid_gather.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, _vp]
+_lib.scan2d_grid_gather.restype = _i
+_lib.scan2d_fwd_wsi.argtypes = [_vp] * 9 + [_i, _i, _i, _i, _i, _u, _vp]
+_lib.scan2d_fwd_wsi.restype = _i
 _lib.scan2d_get_device_error.argtypes = [_vp]
 _lib.scan2d_get_device_error.restype = _i
 _lib.scan2d_strerror.argtypes = [_i]
@@ -215,6 +221,55 @@ def scan2d_bwd(x, delta, A, B, C, Dskip, dy, flags=None, workspace=None, stream=
     if rc:
         raise Scan2dError(rc, "scan2d_bwd")
     return g
+
+
+def scan2d_grid_cells(coords, H, W, cell_patch=None, n_skipped=None, stream=None):
+    """Cell map (H*W int32 CUDA tensor) of a bag whose patch k sits at coords[k] = (row, col)
+    (an (npatch, 2) int32 CUDA tensor): the patch index at each cell, -1 where there is none."""
+    torch = _torch()
+    if coords.dtype != torch.int32 or coords.dim() != 2 or coords.shape[1] != 2 or not coords.is_contiguous():
+        raise ValueError("coords must be a contiguous (npatch, 2) int32 tensor")
+    if cell_patch is None:
+        cell_patch = torch.empty(H * W, dtype=torch.int32, device=coords.device)
+    rc = _lib.scan2d_grid_cells(_ptr(coords), coords.shape[0], H, W, _ptr(cell_patch), _ptr(n_skipped),
+                                _stream_handle(stream))
+    if rc:
+        raise Scan2dError(rc, "scan2d_grid_cells")
+    return cell_patch
+
+
+def scan2d_grid_gather(feat, cell_patch, pad, H, W, x=None, stream=None):
+    """x (1, channels, H, W): feat[cell_patch[i*W + j]] at each cell, pad where it is -1."""
+    torch = _torch()
+    npatch, D = feat.shape
+    if x is None:
+        x = torch.empty((1, D, H, W), dtype=feat.dtype, device=feat.device)
+    flags = SCAN2D_BF16 if feat.dtype == torch.bfloat16 else 0
+    rc = _lib.scan2d_grid_gather(_ptr(feat), _ptr(cell_patch), _ptr(pad), _ptr(x), npatch, D, H, W, flags,
+                                 _stream_handle(stream))
+    if rc:
+        raise Scan2dError(rc, "scan2d_grid_gather")
+    return x
+
+
+def scan2d_fwd_wsi(feat, cell_patch, pad, delta, A, B, C, Dskip=None, y=None, flags=None, stream=None):
+    """scan2d_fwd of one map whose x is read from the bag feat (npatch, channels) through the
+    cell map, pad at non-tissue cells; x itself is never written."""
+    torch = _torch()
+    npatch, D = feat.shape
+    _, _, H, W = delta.shape
+    N = A.shape[1]
+    K = B.shape[1] if B.dim() == 5 else 1
+    if flags is None:
+        flags = flags_for(delta.dtype == torch.bfloat16, (1 << K) - 1)
+    out_dtype = torch.float32 if (delta.dtype == torch.float32 or flags & SCAN2D_OUT_F32) else torch.bfloat16
+    if y is None:
+        y = torch.empty((1, D, H, W), dtype=out_dtype, device=delta.device)
+    rc = _lib.scan2d_fwd_wsi(_ptr(feat), _ptr(cell_patch), _ptr(pad), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+                             _ptr(Dskip), _ptr(y), npatch, D, H, W, N, flags, _stream_handle(stream))
+    if rc:
+        raise Scan2dError(rc, "scan2d_fwd_wsi")
+    return y
 
 
 PLAN_FIELDS = ("launches", "grid", "threads", "smem", "nseg", "cols", "wpc", "mode", "ng",

@@ -147,6 +147,25 @@ def test_bwd_workspace_size_and_host_checks(lib):
     assert call(*bad) == m["SCAN2D_E_ALIGN"]
 
 
+def test_grid_host_checks(lib):
+    m = _header_macros()
+    r = lib.raw()
+    assert r.scan2d_grid_cells(P, -1, 8, 8, P, None, None) == m["SCAN2D_E_DIMS"]
+    assert r.scan2d_grid_cells(P, 4, 0, 8, P, None, None) == m["SCAN2D_E_DIMS"]
+    assert r.scan2d_grid_cells(None, 4, 8, 8, P, None, None) == m["SCAN2D_E_NULL"]
+    assert r.scan2d_grid_cells(P, 4, 8, 8, None, None, None) == m["SCAN2D_E_NULL"]
+    assert r.scan2d_grid_cells(P, 4, 8, 8, P + 2, None, None) == m["SCAN2D_E_ALIGN"]
+    assert r.scan2d_grid_gather(P, P, P, P, 4, 8, 8, 8, 0x10, None) == m["SCAN2D_E_FLAGS"]
+    assert r.scan2d_grid_gather(P, P, P, P, 4, 0, 8, 8, 0, None) == m["SCAN2D_E_DIMS"]
+    assert r.scan2d_grid_gather(P, P, None, P, 4, 8, 8, 8, 0, None) == m["SCAN2D_E_NULL"]
+    assert r.scan2d_grid_gather(P + 2, P, P, P, 4, 8, 8, 8, 0, None) == m["SCAN2D_E_ALIGN"]
+    # the fused forward checks the bag's arguments before the scan's
+    args = (P, P, P, P, P, P, P, None, P)
+    assert r.scan2d_fwd_wsi(*args, -1, 4, 8, 8, 4, 0x10, None) == m["SCAN2D_E_DIMS"]
+    assert r.scan2d_fwd_wsi(P, None, P, P, P, P, P, None, P, 3, 4, 8, 8, 4, 0x10, None) == m["SCAN2D_E_NULL"]
+    assert r.scan2d_fwd_wsi(*args, 3, 4, 8, 8, 4, 0x14, None) == m["SCAN2D_E_FLAGS"]
+
+
 def test_valid_call_without_a_gpu_fails_loudly(lib):
     """No CPU fallback: with valid arguments and no usable device the call is an error."""
     import torch

@@ -481,3 +481,31 @@ def test_planted_mistake_is_caught(oracle_mod, tmp_path, name):
         except AssertionError:
             caught.append(pin.__name__)
     assert caught, f"no pin caught the planted mistake {name}"
+
+
+# ----------------------------------------------------------------------------------------
+# the whole-slide grid ("2DMamba 精读", section 四.2, steps 3-4): a worked example typed out
+# by hand, and the round trip through the seeded bag generator
+# ----------------------------------------------------------------------------------------
+def test_wsi_grid_worked_example(oracle_mod):
+    feat = np.array([[1, 2], [3, 4], [5, 6], [7, 8]], dtype=np.float32)
+    coords = np.array([[0, 1], [1, 2], [0, 1], [5, 0]], dtype=np.int32)   # patch 2 repeats a cell,
+    pad = np.array([-1, -2], dtype=np.float32)                            # patch 3 is off the grid
+    x, cell, skipped = oracle_mod.wsi_grid(feat, coords, pad, 2, 3)
+    assert skipped == 1
+    np.testing.assert_array_equal(cell, [-1, 2, -1, -1, -1, 1])
+    want = np.array([[[-1, 5, -1], [-1, -1, 3]],
+                     [[-2, 6, -2], [-2, -2, 4]]], dtype=np.float32)[None]
+    np.testing.assert_array_equal(x, want)
+
+
+def test_wsi_grid_round_trip(oracle_mod):
+    for dtype in ("f32", "bf16"):
+        w = inputs.WORKLOADS["wsi"].scaled(channels=5, H=19, W=26, dtype=dtype)
+        b = inputs.make_wsi_bag(w, 4)
+        x, cell, skipped = oracle_mod.wsi_grid(b["feat"], b["coords"], b["pad"], w.H, w.W)
+        assert skipped == 0
+        np.testing.assert_array_equal(x, b["x"])
+        assert int((cell >= 0).sum()) == b["feat"].shape[0] == int(b["tissue"].sum())
+        # every non-tissue cell holds the token
+        assert np.all(x[0][:, ~b["tissue"]] == b["pad"][:, None])
