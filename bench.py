@@ -5,7 +5,8 @@ the fraction of the kernel's roofline.  One JSON line on rank 0.
                     [--impl ours|reference] [--no-cpu-baseline] [--others] [--pass fwd|bwd]
 
 --pass bwd times the gradients (scan2d_bwd, one call per step) on the same workloads instead;
---pass wsi --workload wsi times the whole-slide path built from a bag of patch features.
+--pass wsi --workload wsi times the whole-slide path built from a bag of patch features;
+--pass proj times the input projections (x -> delta, B, C) and then the scan on their output.
 
 A step is one scan2d_fwd call over one batch of the workload (every step of the path runs
 in it).  N > 1 runs under torchrun, one rank per GPU; the (b, d) maps are independent, so
@@ -526,6 +527,84 @@ def run_wsi(args, w):
     print(json.dumps(line), flush=True)
 
 
+def run_proj(args, w, R: int = 8):
+    """The input projections (scan2d_proj: x -> delta, B, C with the bias and softplus), then
+    the scan on what they wrote.  value = the projections' Gelem/s (batch*D*H*W of delta per
+    second); roofline = the slower of HBM (x read, delta, B, C written once) and the FP32
+    lanes (D*(R + 2N) + D*R FMAs per position)."""
+    import torch
+    from selective_state_space_scan2d_b200 import scan2d
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    d = inputs.make_inputs(w, seed=0)
+    wt = inputs.make_proj_weights(w.channels, w.N, R, seed=0)
+    x = _to_dev(d["x"], torch, device)
+    Wx, Wdt, bdt = (torch.from_numpy(wt[k]).to(device) for k in ("Wx", "Wdt", "bdt"))
+    A = torch.from_numpy(d["A"]).to(device)
+    Dskip = None if d["Dskip"] is None else torch.from_numpy(d["Dskip"]).to(device)
+    delta = torch.empty_like(x)
+    Bm = torch.empty((w.batch, w.N, w.H, w.W), dtype=x.dtype, device=device)
+    Cm = torch.empty_like(Bm)
+    y = torch.empty_like(x)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        total = 0.0
+        with ClockSampler(0) as clk:
+            for _ in range(args.steps):
+                flush.fill_(1)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+                e1.synchronize()
+                total += e0.elapsed_time(e1)
+        return total / args.steps, clk.summary()
+
+    proj = lambda: scan2d.scan2d_proj(x, Wx, Wdt, bdt, w.N, R, delta=delta, B=Bm, C=Cm, stream=stream)
+    proj_ms, clocks = timed(proj)
+    flags = scan2d.flags_for(w.dtype == "bf16", 1)
+
+    def chain():
+        proj()
+        scan2d.scan2d_fwd(x, delta, A, Bm, Cm, Dskip, y=y, flags=flags, stream=stream)
+
+    chain_ms, _ = timed(chain)
+    s = 2 if w.dtype == "bf16" else 4
+    pos = w.batch * w.H * w.W
+    bytes_ = pos * (2 * w.channels + 2 * w.N) * s
+    fmas = pos * (w.channels * (R + 2 * w.N) + w.channels * R)
+    hbm_gbs, hbm_kind, sm_mhz = _peaks()
+    t_hbm = bytes_ / (hbm_gbs * 1e9)
+    t_fp32 = fmas / (SMS * FP32_PER_CLK_SM * sm_mhz * 1e6)
+    if t_hbm >= t_fp32:
+        roof = {"bound": "hbm", "achieved": bytes_ / (proj_ms * 1e-3) / 1e9, "peak": hbm_gbs, "unit": "GB/s",
+                "peak_kind": f"{hbm_kind} copy bandwidth"}
+    else:
+        roof = {"bound": "alu", "unit_of_bound": "fp32", "achieved": fmas / (proj_ms * 1e-3) / 1e9,
+                "peak": SMS * FP32_PER_CLK_SM * sm_mhz * 1e-3, "unit": "GFMA/s",
+                "peak_kind": f"nominal {SMS} SMs x {FP32_PER_CLK_SM}/clk x {sm_mhz:.0f} MHz"}
+    roof.update({"frac": roof["achieved"] / roof["peak"], "traffic": None, "kernel": "k_proj",
+                 "algorithmic_bytes": bytes_, "algorithmic_fma": fmas,
+                 "t_hbm_ms": t_hbm * 1e3, "t_fp32_ms": t_fp32 * 1e3})
+    line = {
+        "metric": "input projections x -> (delta, B, C) Gelem/s (B*D*H*W)", "value": w.elements / (proj_ms * 1e-3) / 1e9,
+        "unit": "Gelem/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": proj_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32" if w.dtype == "f32" else "bf16-in/f32-acc", "data": "synthetic",
+        "config": {**base_config(w, 1), "pass": "proj", "R": R,
+                   "l2": "a 252 MB buffer is written before every timed step"},
+        "roofline": roof, "clocks": clocks, "gpu_launches": args.steps, "e2e": None,
+        "with_scan": {"ms_per_step": chain_ms, "steps": "scan2d_proj + scan2d_fwd",
+                      "value": w.elements / (chain_ms * 1e-3) / 1e9},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -539,7 +618,7 @@ def main():
     ap.add_argument("--override", action="append", default=[], metavar="KEY=INT",
                     help="change batch/channels/H/W of the workload (smaller cases for ncu captures)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer (e2e) leg")
-    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd", "wsi"],
+    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd", "wsi", "proj"],
                     help="bwd: time the gradients (scan2d_bwd); wsi: the whole-slide path from a bag of patches")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -562,6 +641,9 @@ def main():
         return
     if args.which == "wsi":
         run_wsi(args, w)
+        return
+    if args.which == "proj":
+        run_proj(args, w)
         return
 
     import torch

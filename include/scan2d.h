@@ -76,6 +76,7 @@ extern "C" {
 /* ---- limits ---------------------------------------------------------------------- */
 #define SCAN2D_MAX_N    64     /* states per channel                                   */
 #define SCAN2D_BWD_MAX_N 16    /* states per channel of scan2d_bwd                     */
+#define SCAN2D_PROJ_MAX_R 32   /* rank of the delta projection of scan2d_proj           */
 #define SCAN2D_NOALLOC_SCRATCH_BYTES 33554432  /* fixed scratch of scan2d_fwd_noalloc (32 MiB) */
 
 /* ---- error codes ----------------------------------------------------------------- */
@@ -174,6 +175,24 @@ int scan2d_grid_gather(const void *feat, const int *cell_patch, const void *pad,
 int scan2d_fwd_wsi(const void *feat, const int *cell_patch, const void *pad, const void *delta,
                    const float *A, const void *B, const void *C, const float *Dskip, void *y,
                    int npatch, int channels, int H, int W, int N, unsigned flags, void *stream);
+
+/*
+ * scan2d_proj -- the input-dependent scan parameters from x, in the layouts scan2d_fwd reads.
+ * The pages say the selective parameters are set by the current input ("2DMamba 精读", section
+ * 四.4); the projection is read as Mamba's.  Per position p, contracting the channels of x[p]:
+ *     u = Wx x[p]  (R + 2N values),   B[n,p] = u[R+n],   C[n,p] = u[R+N+n],
+ *     delta[d,p] = softplus(sum_r Wdt[d,r] u[r] + bdt[d]),   softplus(z) = log(1 + e^z).
+ *   x      : device (batch, channels, H, W), fp32 or bf16 (SCAN2D_BF16);
+ *   Wx     : device (R + 2N, channels) fp32;  Wdt: device (channels, R) fp32;  bdt: (channels) fp32;
+ *   delta  : device (batch, channels, H, W), element type of x (written);
+ *   B, C   : device (batch, N, H, W), element type of x (written): the K = 1 layout of scan2d_fwd.
+ * Limits: 1 <= R <= SCAN2D_PROJ_MAX_R, 1 <= N <= 16, and the weights must fit in shared memory
+ * (channels * (R + N) floats, padded; 384 channels fit).  fp32 arithmetic.  Asynchronous on
+ * `stream`.  Returns 0, SCAN2D_E_FLAGS / _DIMS / _N / _NULL / _ALIGN / _LAUNCH.
+ */
+int scan2d_proj(const void *x, const float *Wx, const float *Wdt, const float *bdt, void *delta,
+                void *B, void *C, int batch, int channels, int H, int W, int N, int R,
+                unsigned flags, void *stream);
 
 /*
  * scan2d_query_plan -- how scan2d_fwd would run a call of this shape on a B200 (148

@@ -191,5 +191,31 @@ def wsi_grid(feat, coords, pad, H: int, W: int):
     return x, cell.reshape(-1), skipped
 
 
+def softplus(z):
+    """log(1 + e^z), evaluated without overflow."""
+    return np.logaddexp(0.0, z)
+
+
+def proj(x, Wx, Wdt, bdt, N: int, R: int):
+    """The input-dependent parameters of the scan from x (Mamba's selective projection, the
+    reading of "2DMamba 精读", section 四.4: the parameters follow the current input): per
+    position, u = Wx x (R + 2N values), B = u[R:R+N], C = u[R+N:], delta = softplus(Wdt u[:R]
+    + bdt).  x: (batch, D, H, W) float32 or bf16 bits; returns fp64 delta (batch, D, H, W),
+    B and C (batch, N, H, W)."""
+    xf = np.asarray(x)
+    if xf.dtype == np.uint16:
+        xf = (xf.astype(np.uint32) << 16).view(np.float32)
+    xf = xf.astype(np.float64)
+    batch, D, H, W = xf.shape
+    Wx = np.asarray(Wx, dtype=np.float64)
+    Wdt = np.asarray(Wdt, dtype=np.float64)
+    bdt = np.asarray(bdt, dtype=np.float64)
+    if Wx.shape != (R + 2 * N, D) or Wdt.shape != (D, R) or bdt.shape != (D,):
+        raise ValueError("weights must be Wx (R + 2N, D), Wdt (D, R), bdt (D,)")
+    u = np.einsum("jd,bdhw->bjhw", Wx, xf)
+    z = np.einsum("dr,brhw->bdhw", Wdt, u[:, :R]) + bdt[None, :, None, None]
+    return softplus(z), u[:, R:R + N].copy(), u[:, R + N:].copy()
+
+
 def version() -> int:
     return _load().scan2d_oracle_version()

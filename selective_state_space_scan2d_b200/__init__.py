@@ -11,6 +11,7 @@ _BINDING_NAMES = {
     "SCAN2D_OR_BR", "scan2d_fwd_noalloc", "SCAN2D_E_SCRATCH", "SCAN2D_NOALLOC_SCRATCH_BYTES",
     "SCAN2D_VFIRST", "scan2d_bwd", "scan2d_bwd_workspace_bytes", "SCAN2D_E_WORKSPACE",
     "SCAN2D_BWD_MAX_N", "scan2d_grid_cells", "scan2d_grid_gather", "scan2d_fwd_wsi",
+    "scan2d_proj", "SCAN2D_PROJ_MAX_R",
 }
 
 

@@ -19,6 +19,7 @@ UNITS = {
     os.path.join(HERE, "csrc", "scan2d.cu"): [os.path.join(HERE, "csrc", "scan2d_kernels.cuh"), HEADER],
     os.path.join(HERE, "csrc", "scan2d_bwd.cu"): [HEADER],
     os.path.join(HERE, "csrc", "scan2d_grid.cu"): [HEADER],
+    os.path.join(HERE, "csrc", "scan2d_proj.cu"): [HEADER],
 }
 SOURCES = list(UNITS)
 DEPS = SOURCES + sorted({d for deps in UNITS.values() for d in deps})

@@ -28,7 +28,7 @@ import numpy as np
 ORIENT_TL, ORIENT_TR, ORIENT_BL, ORIENT_BR = 1, 2, 4, 8
 
 _TENSOR_ID = {"x": 1, "delta": 2, "B": 3, "C": 4, "Dskip": 5, "pad": 6, "mask": 7, "A": 8, "dy": 9,
-              "order": 10}
+              "order": 10, "Wx": 11, "Wdt": 12, "bdt": 13}
 
 
 @dataclasses.dataclass(frozen=True)
@@ -186,3 +186,14 @@ def make_wsi_bag(w: Workload | str, seed: int = 0) -> dict:
     if w.dtype == "bf16":
         pad = f32_to_bf16_bits(pad)
     return dict(d, feat=feat, coords=coords, pad=pad, tissue=~mask)
+
+
+def make_proj_weights(channels: int, N: int, R: int, seed: int = 0) -> dict:
+    """Weights of the input projections: Wx (R + 2N, channels) ~ N(0, 1/channels), Wdt
+    (channels, R) ~ N(0, 1/R), and bdt = log(e^dt - 1) with dt = exp(U(log 1e-3, log 1e-1)), so
+    that delta starts near the step sizes of the other workloads.  All float32."""
+    Wx = _rng(seed, "Wx").standard_normal((R + 2 * N, channels), dtype=np.float32) / np.float32(np.sqrt(channels))
+    Wdt = _rng(seed, "Wdt").standard_normal((channels, R), dtype=np.float32) / np.float32(np.sqrt(R))
+    dt = np.exp(np.log(1e-3) + (np.log(1e-1) - np.log(1e-3)) * _rng(seed, "bdt").random(channels))
+    bdt = np.log(np.expm1(dt)).astype(np.float32)
+    return dict(Wx=np.ascontiguousarray(Wx), Wdt=np.ascontiguousarray(Wdt), bdt=bdt, R=R)

@@ -46,6 +46,8 @@ _lib.scan2d_grid_gather.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, _vp]
 _lib.scan2d_grid_gather.restype = _i
 _lib.scan2d_fwd_wsi.argtypes = [_vp] * 9 + [_i, _i, _i, _i, _i, _u, _vp]
 _lib.scan2d_fwd_wsi.restype = _i
+_lib.scan2d_proj.argtypes = [_vp] * 7 + [_i, _i, _i, _i, _i, _i, _u, _vp]
+_lib.scan2d_proj.restype = _i
 _lib.scan2d_get_device_error.argtypes = [_vp]
 _lib.scan2d_get_device_error.restype = _i
 _lib.scan2d_strerror.argtypes = [_i]
@@ -65,6 +67,7 @@ SCAN2D_E_SCRATCH = -11
 SCAN2D_E_WORKSPACE = -12
 SCAN2D_NOALLOC_SCRATCH_BYTES = 32 << 20
 SCAN2D_BWD_MAX_N = 16
+SCAN2D_PROJ_MAX_R = 32
 
 
 class Scan2dError(RuntimeError):
@@ -270,6 +273,26 @@ def scan2d_fwd_wsi(feat, cell_patch, pad, delta, A, B, C, Dskip=None, y=None, fl
     if rc:
         raise Scan2dError(rc, "scan2d_fwd_wsi")
     return y
+
+
+def scan2d_proj(x, Wx, Wdt, bdt, N, R, delta=None, B=None, C=None, stream=None):
+    """delta (like x), B and C ((batch, N, H, W), x's dtype) from x and the projection weights
+    Wx (R + 2N, channels), Wdt (channels, R), bdt (channels,), all CUDA tensors."""
+    torch = _torch()
+    batch, D, H, W = x.shape
+    dev = x.device
+    if delta is None:
+        delta = torch.empty_like(x)
+    if B is None:
+        B = torch.empty((batch, N, H, W), dtype=x.dtype, device=dev)
+    if C is None:
+        C = torch.empty((batch, N, H, W), dtype=x.dtype, device=dev)
+    flags = SCAN2D_BF16 if x.dtype == torch.bfloat16 else 0
+    rc = _lib.scan2d_proj(_ptr(x), _ptr(Wx), _ptr(Wdt), _ptr(bdt), _ptr(delta), _ptr(B), _ptr(C),
+                          batch, D, H, W, N, R, flags, _stream_handle(stream))
+    if rc:
+        raise Scan2dError(rc, "scan2d_proj")
+    return delta, B, C
 
 
 PLAN_FIELDS = ("launches", "grid", "threads", "smem", "nseg", "cols", "wpc", "mode", "ng",

@@ -166,6 +166,24 @@ def test_grid_host_checks(lib):
     assert r.scan2d_fwd_wsi(*args, 3, 4, 8, 8, 4, 0x14, None) == m["SCAN2D_E_FLAGS"]
 
 
+def test_proj_host_checks(lib):
+    m = _header_macros()
+    assert lib.SCAN2D_PROJ_MAX_R == m["SCAN2D_PROJ_MAX_R"]
+    r = lib.raw()
+    ptrs = [P] * 7
+    assert r.scan2d_proj(*ptrs, 1, 8, 4, 4, 4, 2, 0x10, None) == m["SCAN2D_E_FLAGS"]
+    assert r.scan2d_proj(*ptrs, 1, 8, 4, 4, 17, 2, 0, None) == m["SCAN2D_E_N"]
+    assert r.scan2d_proj(*ptrs, 1, 8, 4, 4, 4, 33, 0, None) == m["SCAN2D_E_DIMS"]
+    assert r.scan2d_proj(*ptrs, 0, 8, 4, 4, 4, 2, 0, None) == m["SCAN2D_E_DIMS"]
+    for k in range(7):
+        bad = list(ptrs)
+        bad[k] = None
+        assert r.scan2d_proj(*bad, 1, 8, 4, 4, 4, 2, 0, None) == m["SCAN2D_E_NULL"], k
+    bad = list(ptrs)
+    bad[1] = P + 2
+    assert r.scan2d_proj(*bad, 1, 8, 4, 4, 4, 2, 0, None) == m["SCAN2D_E_ALIGN"]
+
+
 def test_valid_call_without_a_gpu_fails_loudly(lib):
     """No CPU fallback: with valid arguments and no usable device the call is an error."""
     import torch

@@ -509,3 +509,47 @@ def test_wsi_grid_round_trip(oracle_mod):
         assert int((cell >= 0).sum()) == b["feat"].shape[0] == int(b["tissue"].sum())
         # every non-tissue cell holds the token
         assert np.all(x[0][:, ~b["tissue"]] == b["pad"][:, None])
+
+
+# ----------------------------------------------------------------------------------------
+# input projections (reading of "2DMamba 精读", section 四.4): special cases with closed forms
+# and a second library route (torch)
+# ----------------------------------------------------------------------------------------
+def test_proj_special_cases(oracle_mod):
+    import math
+    rng = np.random.default_rng(5)
+    D, N, R = 6, 3, 2
+    x = rng.standard_normal((2, D, 3, 4)).astype(np.float32)
+    bdt = np.array([-3.0, -1.0, 0.0, 0.5, 2.0, 30.0], np.float32)
+    # Wdt = 0: delta is softplus(bdt) everywhere; softplus(0) = ln 2 and softplus(30) ~ 30
+    Wx = rng.standard_normal((R + 2 * N, D)).astype(np.float32)
+    delta, B, C = oracle_mod.proj(x, Wx, np.zeros((D, R), np.float32), bdt, N, R)
+    for d in range(D):
+        want = math.log1p(math.exp(float(bdt[d])))
+        np.testing.assert_allclose(delta[:, d], want, rtol=1e-15, atol=0)
+    assert abs(oracle_mod.softplus(0.0) - math.log(2.0)) < 1e-15
+    # unit rows select channels: B[n] = x[c_n], C[n] = -x[c'_n]
+    Wsel = np.zeros((R + 2 * N, D), np.float32)
+    picks = [4, 0, 5]
+    for n, c in enumerate(picks):
+        Wsel[R + n, c] = 1.0
+        Wsel[R + N + n, (c + 1) % D] = -1.0
+    _, B, C = oracle_mod.proj(x, Wsel, np.zeros((D, R), np.float32), bdt, N, R)
+    for n, c in enumerate(picks):
+        np.testing.assert_array_equal(B[:, n], x[:, c].astype(np.float64))
+        np.testing.assert_array_equal(C[:, n], -x[:, (c + 1) % D].astype(np.float64))
+
+
+def test_proj_against_torch(oracle_mod):
+    import torch
+    rng = np.random.default_rng(6)
+    D, N, R = 10, 4, 3
+    x = rng.standard_normal((2, D, 5, 7)).astype(np.float32)
+    w = inputs.make_proj_weights(D, N, R, seed=2)
+    delta, B, C = oracle_mod.proj(x, w["Wx"], w["Wdt"], w["bdt"], N, R)
+    xt = torch.tensor(x, dtype=torch.float64).permute(0, 2, 3, 1)          # (b, h, w, D)
+    u = xt @ torch.tensor(w["Wx"], dtype=torch.float64).T                   # (b, h, w, R + 2N)
+    z = u[..., :R] @ torch.tensor(w["Wdt"], dtype=torch.float64).T + torch.tensor(w["bdt"], dtype=torch.float64)
+    np.testing.assert_allclose(delta, torch.nn.functional.softplus(z).permute(0, 3, 1, 2).numpy(), rtol=1e-12)
+    np.testing.assert_allclose(B, u[..., R:R + N].permute(0, 3, 1, 2).numpy(), rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(C, u[..., R + N:].permute(0, 3, 1, 2).numpy(), rtol=1e-12, atol=1e-14)
