@@ -75,6 +75,7 @@ struct Variant {
   // [scan order: 0 horizontal first, 1 vertical first]
   KernelFn fn_tma[2], fn_plain[2];
   KernelFn fn_tma16[2], fn_plain16[2];   // up to 16 warps per block (one channel per lane only)
+  KernelFn fn_plain_gx[2], fn_plain16_gx[2];   // plain staging with x read from a bag of patches
 };
 
 template <typename Tin, int NG, int G, int CMAX>
@@ -85,12 +86,17 @@ Variant make_variant() {
             static_cast<size_t>(LP::CARRY_SLOT_BYTES),
             {scan2d_kernel<Tin, NG, G, CMAX, true, kMaxWarps, false>, scan2d_kernel<Tin, NG, G, CMAX, true, kMaxWarps, true>},
             {scan2d_kernel<Tin, NG, G, CMAX, false, kMaxWarps, false>, scan2d_kernel<Tin, NG, G, CMAX, false, kMaxWarps, true>},
-            {nullptr, nullptr}, {nullptr, nullptr}};
+            {nullptr, nullptr}, {nullptr, nullptr},
+            {scan2d_kernel<Tin, NG, G, CMAX, false, kMaxWarps, false, true>,
+             scan2d_kernel<Tin, NG, G, CMAX, false, kMaxWarps, true, true>},
+            {nullptr, nullptr}};
   if constexpr (G == 1) {
     v.fn_tma16[0] = scan2d_kernel<Tin, NG, G, CMAX, true, kMaxWarpsSplit, false>;
     v.fn_tma16[1] = scan2d_kernel<Tin, NG, G, CMAX, true, kMaxWarpsSplit, true>;
     v.fn_plain16[0] = scan2d_kernel<Tin, NG, G, CMAX, false, kMaxWarpsSplit, false>;
     v.fn_plain16[1] = scan2d_kernel<Tin, NG, G, CMAX, false, kMaxWarpsSplit, true>;
+    v.fn_plain16_gx[0] = scan2d_kernel<Tin, NG, G, CMAX, false, kMaxWarpsSplit, false, true>;
+    v.fn_plain16_gx[1] = scan2d_kernel<Tin, NG, G, CMAX, false, kMaxWarpsSplit, true, true>;
   }
   return v;
 }
@@ -483,8 +489,10 @@ int forward(const void* x, const void* delta, const float* A, const void* B, con
     cp = plan_call(s, tma, false, nsm);
   const Plan& pl = cp.pl;
   const int vf = s.vfirst ? 1 : 0;
-  const KernelFn fn = cp.orient_split > 1 ? (tma ? pl.var.fn_tma16[vf] : pl.var.fn_plain16[vf])
-                                         : (tma ? pl.var.fn_tma[vf] : pl.var.fn_plain[vf]);
+  const bool gx = cell_patch != nullptr;
+  const KernelFn fn = cp.orient_split > 1
+                          ? (tma ? pl.var.fn_tma16[vf] : (gx ? pl.var.fn_plain16_gx[vf] : pl.var.fn_plain16[vf]))
+                          : (tma ? pl.var.fn_tma[vf] : (gx ? pl.var.fn_plain_gx[vf] : pl.var.fn_plain[vf]));
 
   Params prm;
   std::memset(&prm, 0, sizeof prm);

@@ -416,7 +416,7 @@ __host__ __device__ constexpr size_t carry_ring_bytes(int warps) {
 }
 
 // ---- the kernel ------------------------------------------------------------------------------
-template <typename Tin, int NG, int G, int CMAX, bool TMA, int MAXW = kMaxWarps, bool VF = false>
+template <typename Tin, int NG, int G, int CMAX, bool TMA, int MAXW = kMaxWarps, bool VF = false, bool GX = false>
 __global__ void __launch_bounds__(MAXW * 32, 1)
 scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps tm) {
   constexpr int R = TMA ? kTileRows : 1;                     // rows per staged tile
@@ -590,7 +590,7 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
         if (region < 2) {
           const int d = grp * L::CPW + rr;
           if (d < p.channels) {
-            if (region == 0 && p.cell_patch != nullptr) {
+            if (GX && region == 0) {                      // GX: x read from a bag
               // x read from the bag through the cell map (one map, b = 0)
               const int kp = __ldg(p.cell_patch + static_cast<size_t>(i) * W + col);
               val = load_raw((kp >= 0 && kp < p.npatch
