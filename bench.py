@@ -124,11 +124,18 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "scan2d_dram_traffic.txt")
 
 
 def kernel_source_hash() -> str:
+    """Hash of the forward's sources with comments and blank lines removed, so that the
+    recorded DRAM traffic stays attached to the code it was measured on."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        text = "\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip())
+        h.update(text.encode())
     return h.hexdigest()[:16]
 
 

@@ -522,7 +522,7 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   if (lane == 0 && is_compute) {
 #pragma unroll
     for (int s = 0; s < DEPTH; ++s) {
-      mbar_init(&s_tfull[warp][s], 1);        // lane 0's expect_tx arrival + the bytes
+      mbar_init(&s_tfull[warp][s], 1);        // the elected lane's expect_tx arrival + the bytes
     }
 #pragma unroll
     for (int s = 0; s < kCarryRing; ++s) {
@@ -613,7 +613,7 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   bool aborted = false;
   if (!TMA && strip_ok) plain_load(0);
 
-  // ---- TMA: lane 0 stages the tiles of this warp's walk, DEPTH tiles ahead -----------------
+  // ---- TMA: the warp stages the tiles of its walk, DEPTH tiles ahead (one elected lane issues) ---
   // A tile is R consecutive scan rows of one orientation (the last one may reach past the map:
   // TMA fills those rows with zeros).  Walk tile wt goes to slot wt % DEPTH; the warp refills
   // a slot right after all its lanes have read the tile's last row.  Once a wait of this warp
@@ -622,7 +622,7 @@ scan2d_kernel(const __grid_constant__ Params p, const __grid_constant__ TmaMaps 
   const int UT = n_or * TPO;                                 // tiles of the walk
   int staged = 0;                                            // tiles of the walk staged so far
   // the next tile to stage, as (orientation, tile in it), with that orientation's stored strip
-  // column, flip and B/C index (lane 0's copy is the one in use)
+  // column, flip and B/C index (every lane keeps the same copy)
   int st_oi = oi_first, st_tr = 0, st_col = 0, st_flip = 0, st_bk = 0;
   auto st_orientation = [&]() {
     const int o = p.orient_code[st_oi];
