@@ -102,14 +102,25 @@ struct Task {
   bool act;
 };
 
-__device__ __forceinline__ bool decode(const Args& p, Task& t) {
+// Warps of one block take adjacent channel groups of one strip (strips_first = false: they
+// share B and C rows and write adjacent blocks of the workspace), or adjacent strips of one
+// channel group (strips_first = true: warps running together add dB and dC at different
+// places).
+__device__ __forceinline__ bool decode(const Args& p, Task& t, bool strips_first = false) {
   const long long task = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
   if (task >= p.tasks) return false;
   const int lane = threadIdx.x & 31;
-  t.cgi = static_cast<int>(task % p.ncg);
-  const long long rest = task / p.ncg;
-  t.s = static_cast<int>(rest % p.S);
-  t.b = static_cast<int>(rest / p.S);
+  if (strips_first) {
+    t.s = static_cast<int>(task % p.S);
+    const long long rest = task / p.S;
+    t.cgi = static_cast<int>(rest % p.ncg);
+    t.b = static_cast<int>(rest / p.ncg);
+  } else {
+    t.cgi = static_cast<int>(task % p.ncg);
+    const long long rest = task / p.ncg;
+    t.s = static_cast<int>(rest % p.S);
+    t.b = static_cast<int>(rest / p.S);
+  }
   t.d = t.cgi * kCh + (lane >> 2);
   t.q = lane & 3;
   t.j0 = t.s * kCols;
@@ -469,7 +480,7 @@ template <typename Tin, typename Tg, int NG, bool FW>
 __global__ void __launch_bounds__(kWarps * 32) k_main(const Args p) {
   extern __shared__ __align__(16) float smem[];
   Task t;
-  if (!decode(p, t)) return;
+  if (!decode(p, t, true)) return;
   const int lane = threadIdx.x & 31, cg = lane >> 2;
   const bool hi = lane & 16, m8 = lane & 8, m4 = lane & 4, m2 = lane & 2, m1 = lane & 1;
   float* buf0 = smem + (threadIdx.x >> 5) * 2 * kBufMain;
