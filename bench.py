@@ -465,8 +465,11 @@ def run_wsi(args, w):
     from selective_state_space_scan2d_b200 import scan2d
     if w.name != "wsi" and not w.wsi_mask:
         raise SystemExit("--pass wsi needs a whole-slide workload (--workload wsi)")
-    torch.cuda.set_device(0)
-    device = torch.device("cuda", 0)
+    if int(os.environ.get("RANK", "0")) != 0:
+        return                       # a one-GPU measurement: under torchrun only rank 0 runs it
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
     b = inputs.make_wsi_bag(w, seed=0)
     t = {k: _to_dev(b[k], torch, device) for k in ("delta", "A", "B", "C", "Dskip", "feat", "pad")}
     coords = torch.from_numpy(b["coords"]).to(device)
@@ -484,7 +487,7 @@ def run_wsi(args, w):
             fn()
         torch.cuda.synchronize()
         total = 0.0
-        with ClockSampler(0) as clk:
+        with ClockSampler(device.index) as clk:
             for _ in range(args.steps):
                 flush.fill_(1)
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -541,8 +544,11 @@ def run_proj(args, w, R: int = 8):
     lanes (D*(R + 2N) + D*R FMAs per position)."""
     import torch
     from selective_state_space_scan2d_b200 import scan2d
-    torch.cuda.set_device(0)
-    device = torch.device("cuda", 0)
+    if int(os.environ.get("RANK", "0")) != 0:
+        return                       # a one-GPU measurement: under torchrun only rank 0 runs it
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
     d = inputs.make_inputs(w, seed=0)
     wt = inputs.make_proj_weights(w.channels, w.N, R, seed=0)
     x = _to_dev(d["x"], torch, device)
@@ -561,7 +567,7 @@ def run_proj(args, w, R: int = 8):
             fn()
         torch.cuda.synchronize()
         total = 0.0
-        with ClockSampler(0) as clk:
+        with ClockSampler(device.index) as clk:
             for _ in range(args.steps):
                 flush.fill_(1)
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
