@@ -252,8 +252,9 @@ int scan2d_fwd_host(const void *x, const void *delta, const float *A, const void
  *                    256-byte aligned, owned by the caller; its contents on entry do not
  *                    matter and are left undefined.  It holds the forward's vertical state of
  *                    one orientation (N floats per element) and the strip carries.
- * Limits: 1 <= N <= SCAN2D_BWD_MAX_N; the default (horizontal-first) scan order only
- * (SCAN2D_VFIRST returns SCAN2D_E_FLAGS).  Asynchronous on `stream`; outputs must not alias
+ * With SCAN2D_VFIRST these are the gradients of the vertical-first forward (the roles of the
+ * two scans swap: the horizontal adjoint reads C*dy, the vertical one adds it up the column).
+ * Limits: 1 <= N <= SCAN2D_BWD_MAX_N.  Asynchronous on `stream`; outputs must not alias
  * inputs or each other.  dA, dB, dC and dDskip are sums built with atomic additions, so their
  * last bits may vary between calls.
  * Returns 0, or SCAN2D_E_NULL / _DIMS / _N / _FLAGS / _ALIGN / _WORKSPACE / _LAUNCH / _DEVICE.

@@ -28,6 +28,9 @@
 //   3. k_states walks each strip's rows forwards from the known carries and stores h.
 //   4. k_main   walks each strip's rows backwards from the known carries, with h of the row
 //               before read back, and produces every gradient.
+// With the vertical-first order the forward's first scan needs no carry and the adjoint's
+// horizontal scan reads only C*dy, so k_states_vf (rows forwards) stores vv and writes both
+// chains' strip terms, then k_carry and k_main as above: three kernels.
 // A warp owns a strip of 8 columns and 8 channels; lane = (channel cg = lane>>2) x (state group
 // q = lane&3), lane q holding states q, q+4, q+8, q+12.  Per-element gradients are summed over
 // a channel's 4 lanes with a shuffle reduce-scatter; dB and dC over the warp's 8 channels, then
@@ -453,6 +456,90 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_states(const Args p) {
   }
 }
 
+// ---- 3'. vertical-first order: the forward's vertical state and both carry terms ---------------
+// In this order the forward's first (vertical) scan needs no carry and the adjoint's horizontal
+// scan reads only C*dy, so one pass down the rows stores vv and writes the strip terms of both
+// horizontal chains (the forward one over vv, the adjoint one over C*dy) and the product of Abar.
+template <typename Tin, typename Tg, int NG, bool FW>
+__global__ void __launch_bounds__(kWarps * 32, 2) k_states_vf(const Args p) {
+  extern __shared__ __align__(16) float smem[];
+  Task t;
+  if (!decode(p, t)) return;
+  const int lane = threadIdx.x & 31, cg = lane >> 2;
+  float* buf0 = smem + (threadIdx.x >> 5) * 2 * kBufStates;
+  float A2[NG];
+  bool nok[NG];
+#pragma unroll
+  for (int g = 0; g < NG; ++g) {
+    const int n = t.q + 4 * g;
+    nok[g] = n < p.N;
+    A2[g] = (t.act && nok[g]) ? p.A[(size_t)t.d * p.N + n] * kLog2e : 0.f;
+  }
+  float2 vv[NG][kPairs];
+#pragma unroll
+  for (int g = 0; g < NG; ++g)
+#pragma unroll
+    for (int k = 0; k < kPairs; ++k) vv[g][k] = make_float2(0.f, 0.f);
+
+  InputPrefetch<Tin, Tg, NG, true, true> pf;
+  pf.init(p, t, lane);
+  pf.load(p, row_of(p, 0));
+  pf.store(buf0, lane);
+  __syncwarp();
+  for (int ii = 0; ii < p.H; ++ii) {
+    const int i = row_of(p, ii);
+    float* cur = buf0 + (ii & 1) * kBufStates;
+    float* nxt = buf0 + ((ii + 1) & 1) * kBufStates;
+    if (ii + 1 < p.H) pf.load(p, row_of(p, ii + 1));
+    float2 xv[kPairs], dl[kPairs], gy[kPairs], dxp[kPairs];
+    lds8x2(cur + kOffX + cg * kCols, xv);
+    lds8x2(cur + kOffD + cg * kCols, dl);
+    lds8x2(cur + kOffG + cg * kCols, gy);
+#pragma unroll
+    for (int k = 0; k < kPairs; ++k) dxp[k] = __fmul2_rn(dl[k], xv[k]);
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+      const int n = t.q + 4 * g;
+      float2 bv[kPairs], cv[kPairs], a[kPairs], aw[kPairs];
+      lds8x2(cur + kOffB + n * kCols, bv);
+      lds8x2(cur + kOffC + n * kCols, cv);
+      const float2 A2g = make_float2(A2[g], A2[g]);
+      float2 prod2 = make_float2(1.f, 1.f);
+#pragma unroll
+      for (int k = 0; k < kPairs; ++k) {
+        const float2 arg = __fmul2_rn(dl[k], A2g);
+        a[k] = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+        prod2 = __fmul2_rn(prod2, a[k]);
+        vv[g][k] = __ffma2_rn(a[k], vv[g][k], __fmul2_rn(dxp[k], bv[k]));   // vertical, first
+        aw[k] = __fmul2_rn(a[k], __fmul2_rn(cv[k], gy[k]));                // Abar*C*dy
+      }
+      float r = 0.f;                          // forward: h leaving the strip, from zero
+#pragma unroll
+      for (int k = 0; k < kCols; ++k) {
+        const int c = FW ? kCols - 1 - k : k;
+        r = fmaf(lo_hi(a, c), r, lo_hi(vv[g], c));
+      }
+      float hc = 0.f;                         // adjoint: Abar*g2 leaving the strip, from zero
+#pragma unroll
+      for (int k = 0; k < kCols; ++k) {
+        const int c = FW ? k : kCols - 1 - k;
+        hc = fmaf(lo_hi(a, c), hc, lo_hi(aw, c));
+      }
+      if (t.act && nok[g]) {
+        float* dst = p.hsave + hs_idx(p, t.b, t.d, i, t.s, n);
+        *reinterpret_cast<float4*>(dst) = make_float4(vv[g][0].x, vv[g][0].y, vv[g][1].x, vv[g][1].y);
+        *reinterpret_cast<float4*>(dst + 4) = make_float4(vv[g][2].x, vv[g][2].y, vv[g][3].x, vv[g][3].y);
+        const size_t ci = carry_idx(p, t.b, t.d, i, t.s, n);
+        p.tf[ci] = r;
+        p.tb[ci] = hc;
+        p.beta[ci] = prod2.x * prod2.y;
+      }
+    }
+    if (ii + 1 < p.H) pf.store(nxt, lane);
+    __syncwarp();
+  }
+}
+
 // ---- 4. gradients -------------------------------------------------------------------------------
 template <typename Tg>
 __device__ __forceinline__ void put2(Tg* out, size_t idx, float v0, float v1, bool ok0, bool ok1, bool vec) {
@@ -476,7 +563,7 @@ __device__ __forceinline__ void put2(Tg* out, size_t idx, float v0, float v1, bo
   }
 }
 
-template <typename Tin, typename Tg, int NG, bool FW>
+template <typename Tin, typename Tg, int NG, bool FW, bool VF = false>
 __global__ void __launch_bounds__(kWarps * 32) k_main(const Args p) {
   extern __shared__ __align__(16) float smem[];
   Task t;
@@ -570,6 +657,8 @@ __global__ void __launch_bounds__(kWarps * 32) k_main(const Args p) {
       const float cin = live ? cur[kOffCB + cg * p.N + n] : 0.f;
       const float2 A2g = make_float2(A2[g], A2[g]);
       const float2 Afg = make_float2(Af[g], Af[g]);
+      float pB[kCols], pC[kCols];
+      if constexpr (!VF) {
       float2 a[kPairs], u[kPairs], gh[kPairs];
 #pragma unroll
       for (int k = 0; k < kPairs; ++k) {
@@ -595,7 +684,6 @@ __global__ void __launch_bounds__(kWarps * 32) k_main(const Args p) {
         if (c & 1) cpre[c >> 1].y = carry; else cpre[c >> 1].x = carry;
         carry = fmaf(lo_hi(a, c), carry, lo_hi(V[g], c));  // a*(gh + carry)
       }
-      float pB[kCols], pC[kCols];
 #pragma unroll
       for (int k = 0; k < kPairs; ++k) {       // what each column adds
         const float2 hc = __ffma2_rn(a[k], hp[k], rr[k]);   // h of this row
@@ -608,6 +696,49 @@ __global__ void __launch_bounds__(kWarps * 32) k_main(const Args p) {
         const float2 c2 = __fmul2_rn(gy[k], hc);
         pB[2 * k] = b2.x; pB[2 * k + 1] = b2.y;
         pC[2 * k] = c2.x; pC[2 * k + 1] = c2.y;
+      }
+      } else {
+      // vertical first: hp holds vv of the row before; g2 is the adjoint of the horizontal
+      // (second) scan, g1 that of the vertical (first) scan, carried up the column in V
+      float2 a[kPairs], vvc[kPairs], w[kPairs], aw[kPairs];
+#pragma unroll
+      for (int k = 0; k < kPairs; ++k) {
+        const float2 arg = __fmul2_rn(dl[k], A2g);
+        a[k] = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+        vvc[k] = __ffma2_rn(a[k], hp[k], __fmul2_rn(dxp[k], bv[k]));   // vv of this row
+        w[k] = __fmul2_rn(cv[k], gy[k]);
+        aw[k] = __fmul2_rn(a[k], w[k]);
+      }
+      float2 hhp[kPairs], hcur[kPairs], cpre[kPairs];
+      float r = hin;
+#pragma unroll
+      for (int k = 0; k < kCols; ++k) {       // forward recompute: h before and after each column
+        const int c = FW ? kCols - 1 - k : k;
+        if (c & 1) hhp[c >> 1].y = r; else hhp[c >> 1].x = r;
+        r = fmaf(lo_hi(a, c), r, lo_hi(vvc, c));
+        if (c & 1) hcur[c >> 1].y = r; else hcur[c >> 1].x = r;
+      }
+      float carry = cin;
+#pragma unroll
+      for (int k = 0; k < kCols; ++k) {       // adjoint, horizontal: carry before each column
+        const int c = FW ? k : kCols - 1 - k;
+        if (c & 1) cpre[c >> 1].y = carry; else cpre[c >> 1].x = carry;
+        carry = fmaf(lo_hi(a, c), carry, lo_hi(aw, c));    // a*(C*dy + carry)
+      }
+#pragma unroll
+      for (int k = 0; k < kPairs; ++k) {       // what each column adds
+        const float2 g2 = __fadd2_rn(w[k], cpre[k]);
+        const float2 g1 = __fadd2_rn(g2, V[g][k]);
+        V[g][k] = __fmul2_rn(a[k], g1);                      // adjoint, vertical, carried up
+        const float2 ta = __fmul2_rn(__ffma2_rn(g2, hhp[k], __fmul2_rn(g1, hp[k])), a[k]);
+        s1[k] = __ffma2_rn(g1, bv[k], s1[k]);
+        s2[k] = __ffma2_rn(ta, Afg, s2[k]);
+        dAacc[g] = __ffma2_rn(ta, dl[k], dAacc[g]);
+        const float2 b2 = __fmul2_rn(g1, dxp[k]);
+        const float2 c2 = __fmul2_rn(gy[k], hcur[k]);
+        pB[2 * k] = b2.x; pB[2 * k + 1] = b2.y;
+        pC[2 * k] = c2.x; pC[2 * k + 1] = c2.y;
+      }
       }
       // dB, dC: sum over the warp's 8 channels (lanes xor 16, 8, 4 share the state)
       float k1[kCols];
@@ -700,7 +831,6 @@ int popcount4(unsigned v) { return (v & 1) + ((v >> 1) & 1) + ((v >> 2) & 1) + (
 int bwd_shape(int batch, int channels, int H, int W, int N, unsigned flags, BwdShape* s) {
   if (flags & ~SCAN2D_FLAGS_KNOWN) return SCAN2D_E_FLAGS;
   if ((flags & SCAN2D_OUT_F32) && !(flags & SCAN2D_BF16)) return SCAN2D_E_FLAGS;
-  if (flags & SCAN2D_VFIRST) return SCAN2D_E_FLAGS;
   if (batch < 1 || channels < 1 || H < 1 || W < 1) return SCAN2D_E_DIMS;
   if (N < 1 || N > kMaxNBwd) return SCAN2D_E_N;
   const unsigned long long hw = static_cast<unsigned long long>(H) * W;
@@ -764,16 +894,25 @@ bool launch_warps(K kern, int floats_per_buffer, const Args& a, cudaStream_t st)
 }
 
 template <typename Tin, typename Tg, int NG>
-int launch_orientation(const Args& a, bool fw, cudaStream_t st) {
+int launch_orientation(const Args& a, bool fw, bool vf, cudaStream_t st) {
   const long long threads = (long long)a.batch * a.H * a.ncg * kCh * a.N;
   const unsigned cblocks = static_cast<unsigned>((threads + 255) / 256);
-  bool ok = fw ? launch_warps(k_pre<Tin, Tg, NG, true>, kBufPre, a, st)
-               : launch_warps(k_pre<Tin, Tg, NG, false>, kBufPre, a, st);
-  k_carry<<<cblocks, 256, 0, st>>>(a, fw ? 1 : 0);
-  ok = ok && (fw ? launch_warps(k_states<Tin, NG, true>, kBufStates, a, st)
-                 : launch_warps(k_states<Tin, NG, false>, kBufStates, a, st));
-  ok = ok && (fw ? launch_warps(k_main<Tin, Tg, NG, true>, kBufMain, a, st)
-                 : launch_warps(k_main<Tin, Tg, NG, false>, kBufMain, a, st));
+  bool ok;
+  if (!vf) {                   // horizontal first: terms (rows up), carries, states (rows down), gradients
+    ok = fw ? launch_warps(k_pre<Tin, Tg, NG, true>, kBufPre, a, st)
+            : launch_warps(k_pre<Tin, Tg, NG, false>, kBufPre, a, st);
+    k_carry<<<cblocks, 256, 0, st>>>(a, fw ? 1 : 0);
+    ok = ok && (fw ? launch_warps(k_states<Tin, NG, true>, kBufStates, a, st)
+                   : launch_warps(k_states<Tin, NG, false>, kBufStates, a, st));
+    ok = ok && (fw ? launch_warps(k_main<Tin, Tg, NG, true>, kBufMain, a, st)
+                   : launch_warps(k_main<Tin, Tg, NG, false>, kBufMain, a, st));
+  } else {                     // vertical first: states and terms (rows down), carries, gradients
+    ok = fw ? launch_warps(k_states_vf<Tin, Tg, NG, true>, kBufStates, a, st)
+            : launch_warps(k_states_vf<Tin, Tg, NG, false>, kBufStates, a, st);
+    k_carry<<<cblocks, 256, 0, st>>>(a, fw ? 1 : 0);
+    ok = ok && (fw ? launch_warps(k_main<Tin, Tg, NG, true, true>, kBufMain, a, st)
+                   : launch_warps(k_main<Tin, Tg, NG, false, true>, kBufMain, a, st));
+  }
   if (!ok) {
     cudaGetLastError();
     return SCAN2D_E_LAUNCH;
@@ -782,10 +921,10 @@ int launch_orientation(const Args& a, bool fw, cudaStream_t st) {
 }
 
 template <typename Tin, typename Tg>
-int launch_ng(const Args& a, bool fw, cudaStream_t st) {
-  if (a.N <= 4) return launch_orientation<Tin, Tg, 1>(a, fw, st);
-  if (a.N <= 8) return launch_orientation<Tin, Tg, 2>(a, fw, st);
-  return launch_orientation<Tin, Tg, 4>(a, fw, st);
+int launch_ng(const Args& a, bool fw, bool vf, cudaStream_t st) {
+  if (a.N <= 4) return launch_orientation<Tin, Tg, 1>(a, fw, vf, st);
+  if (a.N <= 8) return launch_orientation<Tin, Tg, 2>(a, fw, vf, st);
+  return launch_orientation<Tin, Tg, 4>(a, fw, vf, st);
 }
 
 }  // namespace
@@ -853,6 +992,7 @@ int scan2d_bwd(const void* x, const void* delta, const float* A, const void* B, 
   a.vec2 = W % 2 == 0 && aligned(dx, 2 * s.out_elem) && aligned(ddelta, 2 * s.out_elem) &&
            aligned(dB, 8) && aligned(dC, 8);
 
+  const bool vf = (flags & SCAN2D_VFIRST) != 0;
   int k = 0;
   for (int o = 0; o < 4; ++o) {
     if (!((s.orient >> o) & 1u)) continue;
@@ -861,9 +1001,9 @@ int scan2d_bwd(const void* x, const void* delta, const float* A, const void* B, 
     a.first = k == 0;
     a.last = k == s.K - 1;
     const bool fw = (o & 1) != 0;
-    if (!s.bf16) rc = launch_ng<float, float>(a, fw, st);
-    else if (s.out_f32) rc = launch_ng<uint16_t, float>(a, fw, st);
-    else rc = launch_ng<uint16_t, uint16_t>(a, fw, st);
+    if (!s.bf16) rc = launch_ng<float, float>(a, fw, vf, st);
+    else if (s.out_f32) rc = launch_ng<uint16_t, float>(a, fw, vf, st);
+    else rc = launch_ng<uint16_t, uint16_t>(a, fw, vf, st);
     if (rc) return rc;
     ++k;
   }

@@ -135,7 +135,7 @@ def test_bwd_workspace_size_and_host_checks(lib):
     call = lambda *ptrs, size=n, flags=0x10, d=dims: r.scan2d_bwd(*ptrs, size, *d, flags, None)
     good = [P] * 14
     good[5] = None                                     # Dskip may be NULL
-    assert call(*good, flags=0x18) == m["SCAN2D_E_FLAGS"]          # vertical-first: forward only
+    assert call(*good, flags=0x14) == m["SCAN2D_E_FLAGS"]          # a reserved bit
     assert call(*good, d=(1, 4, 8, 8, 17)) == m["SCAN2D_E_N"]
     assert call(*good, size=n - 1) == m["SCAN2D_E_WORKSPACE"]
     for k in (0, 6, 7, 13):

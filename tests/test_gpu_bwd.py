@@ -33,7 +33,8 @@ def _dy_f64(dy):
 def _gpu_bwd(d, dy, out_f32=False):
     from selective_state_space_scan2d_b200 import scan2d
     t = to_torch(d)
-    flags = scan2d.flags_for(d["x"].dtype == np.uint16, d["orient_mask"], out_f32=out_f32)
+    flags = scan2d.flags_for(d["x"].dtype == np.uint16, d["orient_mask"], out_f32=out_f32,
+                             vfirst=d.get("vfirst", False))
     g = scan2d.scan2d_bwd(t["x"], t["delta"], t["A"], t["B"], t["C"], t["Dskip"], _dy_torch(dy), flags=flags)
     assert scan2d.scan2d_get_device_error() == 0
     return {k: v.detach().float().cpu().numpy().astype(np.float64) for k, v in g.items()}
@@ -72,7 +73,17 @@ CASES = {
     "f32_h1": ("giga", dict(channels=8, H=1, W=37), False),
     "f32_w1": ("giga", dict(channels=8, H=23, W=1, orient_mask=0b0011), False),
     "f32_wide": ("giga", dict(channels=16, H=6, W=200), False),
+    # the vertical-first scan order
+    "f32_vf_ragged": ("giga", dict(batch=2, channels=12, H=9, W=21, vfirst=True), False),
+    "f32_vf_all4": ("giga", dict(channels=8, H=7, W=16, orient_mask=0xF, vfirst=True), False),
+    "f32_vf_n4_nodskip": ("tiny", dict(channels=9, H=10, W=11, dskip=False, vfirst=True), False),
+    "bf16_vf_vision_like": ("vision", dict(batch=2, channels=16, H=10, W=14, vfirst=True), False),
+    "f32_vf_wide_br": ("giga", dict(channels=16, H=6, W=200, orient_mask=0b1000, vfirst=True), False),
 }
+
+
+def _mask(d):
+    return d["orient_mask"] | (0x10 if d.get("vfirst") else 0)
 
 
 @pytest.mark.parametrize("case", sorted(CASES))
@@ -82,7 +93,7 @@ def test_bwd_parity(oracle_mod, case):
     d = inputs.make_inputs(w, seed=3)
     dy = inputs.make_cotangent(w, seed=3, out_f32=out_f32)
     g = _gpu_bwd(d, dy, out_f32)
-    args = (d["x"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"], _dy_f64(dy), d["orient_mask"])
+    args = (d["x"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"], _dy_f64(dy), _mask(d))
     ref = oracle_mod.scan2d_bwd(*args)
     maj = oracle_mod.scan2d_bwd(*args, majorant=True)
     _check(g, ref, maj, w.dtype == "bf16" and not out_f32, case)
@@ -111,7 +122,7 @@ def test_bwd_repeatable_and_workspace_reused(oracle_mod):
         torch.testing.assert_close(g1[k], g2[k], rtol=1e-5, atol=1e-6)
 
 
-def test_bwd_rejects_small_workspace_and_vfirst():
+def test_bwd_rejects_small_workspace():
     import torch
     from selective_state_space_scan2d_b200 import scan2d
     w = workload("tiny")
@@ -124,9 +135,6 @@ def test_bwd_rejects_small_workspace_and_vfirst():
     with pytest.raises(scan2d.Scan2dError) as e:
         scan2d.scan2d_bwd(t["x"], t["delta"], t["A"], t["B"], t["C"], t["Dskip"], dy, flags=flags, workspace=small)
     assert e.value.code == scan2d.SCAN2D_E_WORKSPACE
-    with pytest.raises(scan2d.Scan2dError):
-        scan2d.scan2d_bwd(t["x"], t["delta"], t["A"], t["B"], t["C"], t["Dskip"], dy,
-                          flags=flags | scan2d.SCAN2D_VFIRST)
 
 
 def _crop(d, rows, cols, channels=None):
