@@ -66,6 +66,17 @@ __global__ void __launch_bounds__(kTile * kRowsY) k_gather(const T* __restrict__
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// an sm_100 device is current (the library is built for it alone)
+int device_ok() {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return SCAN2D_E_DEVICE;
+  }
+  return major == 10 ? SCAN2D_OK : SCAN2D_E_DEVICE;
+}
+
 }  // namespace
 
 extern "C" {
@@ -76,6 +87,7 @@ int scan2d_grid_cells(const int* coords, int npatch, int H, int W, int* cell_pat
     return SCAN2D_E_DIMS;
   if (!cell_patch || (npatch > 0 && !coords)) return SCAN2D_E_NULL;
   if (!aligned(cell_patch, 4) || !aligned(coords, 4) || !aligned(n_skipped, 4)) return SCAN2D_E_ALIGN;
+  if (const int rc = device_ok()) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(cell_patch, 0xFF, (size_t)H * W * sizeof(int), st) != cudaSuccess ||
       (n_skipped && cudaMemsetAsync(n_skipped, 0, sizeof(int), st) != cudaSuccess)) {
@@ -96,6 +108,7 @@ int scan2d_grid_gather(const void* feat, const int* cell_patch, const void* pad,
   if (!cell_patch || !pad || !x || (npatch > 0 && !feat)) return SCAN2D_E_NULL;
   const size_t el = (flags & SCAN2D_BF16) ? 2 : 4;
   if (!aligned(feat, el) || !aligned(pad, el) || !aligned(x, el) || !aligned(cell_patch, 4)) return SCAN2D_E_ALIGN;
+  if (const int rc = device_ok()) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const dim3 grid(static_cast<unsigned>((cells + kTile - 1) / kTile), static_cast<unsigned>((channels + kTile - 1) / kTile));
   const dim3 block(kTile, kRowsY);

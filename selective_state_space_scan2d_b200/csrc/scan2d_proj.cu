@@ -164,6 +164,17 @@ __global__ void __launch_bounds__(kThreads) k_proj(const ProjArgs a) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// an sm_100 device is current (the library is built for it alone)
+int device_ok() {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return SCAN2D_E_DEVICE;
+  }
+  return major == 10 ? SCAN2D_OK : SCAN2D_E_DEVICE;
+}
+
 template <typename T, int RP>
 int launch(const ProjArgs& a, cudaStream_t st) {
   constexpr int NU = RP + 2 * kNB;
@@ -206,6 +217,7 @@ int scan2d_proj(const void* x, const float* Wx, const float* Wdt, const float* b
     return SCAN2D_E_ALIGN;
   const bool pairs = hw % 2 == 0 && aligned(x, 2 * el) && aligned(delta, 2 * el) && aligned(B, 2 * el) &&
                      aligned(C, 2 * el);
+  if (const int rc = device_ok()) return rc;
   ProjArgs a{x, Wx, Wdt, bdt, delta, B, C, batch, channels, static_cast<int>(hw), N, R, pairs ? 1 : 0};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return el == 2 ? launch_r<uint16_t>(a, st) : launch_r<float>(a, st);

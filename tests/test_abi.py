@@ -190,8 +190,14 @@ def test_valid_call_without_a_gpu_fails_loudly(lib):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     m = _header_macros()
-    rc = lib.raw().scan2d_fwd(P, P, P, P, P, None, P, 1, 4, 8, 8, 4, 0x10, None)
-    assert rc == m["SCAN2D_E_DEVICE"]
+    r = lib.raw()
+    assert r.scan2d_fwd(P, P, P, P, P, None, P, 1, 4, 8, 8, 4, 0x10, None) == m["SCAN2D_E_DEVICE"]
+    n = lib.scan2d_bwd_workspace_bytes(1, 4, 8, 8, 4, 0x10)
+    assert r.scan2d_bwd(P, P, P, P, P, None, P, P, P, P, P, P, None, P, n, 1, 4, 8, 8, 4, 0x10, None) == m["SCAN2D_E_DEVICE"]
+    assert r.scan2d_fwd_wsi(P, P, P, P, P, P, P, None, P, 3, 4, 8, 8, 4, 0x10, None) == m["SCAN2D_E_DEVICE"]
+    assert r.scan2d_grid_cells(P, 4, 8, 8, P, None, None) == m["SCAN2D_E_DEVICE"]
+    assert r.scan2d_grid_gather(P, P, P, P, 4, 8, 8, 8, 0, None) == m["SCAN2D_E_DEVICE"]
+    assert r.scan2d_proj(P, P, P, P, P, P, P, 1, 8, 4, 4, 4, 2, 0, None) == m["SCAN2D_E_DEVICE"]
     x = torch.zeros(1, 4, 8, 8)
     with pytest.raises(ValueError):
         lib.scan2d_fwd(x, x, torch.zeros(4, 4), torch.zeros(1, 4, 8, 8), torch.zeros(1, 4, 8, 8))
