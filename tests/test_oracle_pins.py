@@ -553,3 +553,28 @@ def test_proj_against_torch(oracle_mod):
     np.testing.assert_allclose(delta, torch.nn.functional.softplus(z).permute(0, 3, 1, 2).numpy(), rtol=1e-12)
     np.testing.assert_allclose(B, u[..., R:R + N].permute(0, 3, 1, 2).numpy(), rtol=1e-12, atol=1e-14)
     np.testing.assert_allclose(C, u[..., R + N:].permute(0, 3, 1, 2).numpy(), rtol=1e-12, atol=1e-14)
+
+
+def test_bwd_single_cell_closed_form(oracle_mod):
+    """A 1 x 1 map: y = sum_n C_n dt B_n x + D x, so every gradient has a closed form
+    (Abar never multiplies anything, so dA = 0)."""
+    rng = np.random.default_rng(12)
+    N = 3
+    x = rng.standard_normal((1, 1, 1, 1)).astype(np.float32)
+    dt = np.abs(rng.standard_normal((1, 1, 1, 1))).astype(np.float32)
+    A = -rng.random((1, N)).astype(np.float32)
+    B = rng.standard_normal((1, 1, N, 1, 1)).astype(np.float32)
+    C = rng.standard_normal((1, 1, N, 1, 1)).astype(np.float32)
+    D = rng.standard_normal(1).astype(np.float32)
+    dy = rng.standard_normal((1, 1, 1, 1))
+    for mask in (1, 1 | VFIRST):
+        g = oracle_mod.scan2d_bwd(x, dt, A, B, C, D, dy, mask)
+        xs, ds, gys = float(x[0, 0, 0, 0]), float(dt[0, 0, 0, 0]), float(dy[0, 0, 0, 0])
+        Bv = B[0, 0, :, 0, 0].astype(np.float64)
+        Cv = C[0, 0, :, 0, 0].astype(np.float64)
+        np.testing.assert_allclose(g["dx"][0, 0, 0, 0], gys * (ds * np.dot(Bv, Cv) + float(D[0])), rtol=1e-14)
+        np.testing.assert_allclose(g["ddelta"][0, 0, 0, 0], gys * xs * np.dot(Bv, Cv), rtol=1e-14)
+        np.testing.assert_array_equal(g["dA"], 0.0)
+        np.testing.assert_allclose(g["dB"][0, 0, :, 0, 0], gys * Cv * ds * xs, rtol=1e-14)
+        np.testing.assert_allclose(g["dC"][0, 0, :, 0, 0], gys * Bv * ds * xs, rtol=1e-14)
+        np.testing.assert_allclose(g["dDskip"][0], gys * xs, rtol=1e-14)
