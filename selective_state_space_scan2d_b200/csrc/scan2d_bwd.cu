@@ -884,7 +884,9 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 template <typename K>
 bool launch_warps(K kern, int floats_per_buffer, const Args& a, cudaStream_t st) {
-  const unsigned blocks = static_cast<unsigned>((a.tasks + kWarps - 1) / kWarps);
+  const long long nblocks = (a.tasks + kWarps - 1) / kWarps;
+  if (nblocks > 0x7fffffffLL) return false;
+  const unsigned blocks = static_cast<unsigned>(nblocks);
   const size_t smem = static_cast<size_t>(kWarps) * 2 * floats_per_buffer * sizeof(float);
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
@@ -896,6 +898,7 @@ bool launch_warps(K kern, int floats_per_buffer, const Args& a, cudaStream_t st)
 template <typename Tin, typename Tg, int NG>
 int launch_orientation(const Args& a, bool fw, bool vf, cudaStream_t st) {
   const long long threads = (long long)a.batch * a.H * a.ncg * kCh * a.N;
+  if ((threads + 255) / 256 > 0x7fffffffLL) return SCAN2D_E_DIMS;
   const unsigned cblocks = static_cast<unsigned>((threads + 255) / 256);
   bool ok;
   if (!vf) {                   // horizontal first: terms (rows up), carries, states (rows down), gradients
