@@ -78,8 +78,6 @@ struct Args {
   int k;                    // orientation index: B_k, C_k, dB_k, dC_k
   int flipH;
   int first, last;          // first / last orientation of the call
-  int vec_in;               // input rows allow 16-byte loads
-  int vec_g;                // dy rows allow 16-byte loads
   int vec2;                 // W even and outputs aligned: 2-column stores and atomics
 };
 
@@ -143,11 +141,6 @@ __device__ __forceinline__ size_t carry_idx(const Args& p, int b, int d, int i, 
 // first float of the 8 columns of (b, row i, strip s, channel d, state n) in hsave
 __device__ __forceinline__ size_t hs_idx(const Args& p, int b, int d, int i, int s, int n) {
   return carry_idx(p, b, d, i, s, n) * kCols;
-}
-
-__device__ __forceinline__ void st8(float* dst, const float (&v)[kCols]) {
-  *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
-  *reinterpret_cast<float4*>(dst + 4) = make_float4(v[4], v[5], v[6], v[7]);
 }
 
 __device__ __forceinline__ void lds8(const float* src, float (&v)[kCols]) {
@@ -989,9 +982,6 @@ int scan2d_bwd(const void* x, const void* delta, const float* A, const void* B, 
   a.batch = batch; a.channels = channels; a.H = H; a.W = W; a.N = N; a.K = s.K; a.S = s.S;
   a.ncg = s.ncg;
   a.tasks = (long long)batch * s.S * s.ncg;
-  const size_t row_in = (size_t)W * s.in_elem, row_out = (size_t)W * s.out_elem;
-  a.vec_in = row_in % 16 == 0 && aligned(x, 16) && aligned(delta, 16) && aligned(B, 16) && aligned(C, 16);
-  a.vec_g = row_out % 16 == 0 && aligned(dy, 16);
   a.vec2 = W % 2 == 0 && aligned(dx, 2 * s.out_elem) && aligned(ddelta, 2 * s.out_elem) &&
            aligned(dB, 8) && aligned(dC, 8);
 
