@@ -73,6 +73,8 @@ CASES = {
     "f32_h1": ("giga", dict(channels=8, H=1, W=37), False),
     "f32_w1": ("giga", dict(channels=8, H=23, W=1, orient_mask=0b0011), False),
     "f32_wide": ("giga", dict(channels=16, H=6, W=200), False),
+    "f32_n13_odd_states": ("tiny", dict(batch=1, channels=11, N=13, H=7, W=19, orient_mask=0b0101), False),
+    "bf16_n5_odd_states": ("vision", dict(batch=1, channels=8, N=5, H=6, W=12), False),
     # the vertical-first scan order
     "f32_vf_ragged": ("giga", dict(batch=2, channels=12, H=9, W=21, vfirst=True), False),
     "f32_vf_all4": ("giga", dict(channels=8, H=7, W=16, orient_mask=0xF, vfirst=True), False),
